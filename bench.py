@@ -1,0 +1,618 @@
+#!/usr/bin/env python
+"""Benchmark of the fused W4A4 + low-rank linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl twq|reference]
+
+One step is one pass of the hot path over one batch: the online activation
+quantizer (twq_quantize_act) and the fused dual-component layer
+(twq_fused_linear) on inputs already resident in HBM. Steps run from a CUDA
+graph on one stream; the K timed steps are bracketed by a barrier and a device
+synchronize, timed with CUDA events, max over ranks. Packed weights rotate over
+enough copies that consecutive uses of one copy are more than 2x the 126 MB L2
+apart, so weight bytes come from HBM.
+
+Multi-GPU: the layer shards over tokens with replicated weights and no data
+exchange (replicas), so each rank runs the same per-GPU workload ("weak").
+
+Prints one JSON line. With --impl reference the CPU oracle is timed on the host
+cores instead, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOP/s bf16)
+
+WORKLOADS = {
+    # name: (synth workload, batch)
+    "decode16": ("decode", 16),
+    "decode4": ("decode", 4),
+    "decode1": ("decode", 1),
+    "gateup": ("gateup", 2048),
+    "down": ("down", 4096),
+    "large": ("large", 8192),
+    "tiny": ("tiny", 16),
+}
+DEFAULT_WORKLOAD = "decode16"
+SWEEP = ["decode1", "decode4", "gateup", "down", "large"]
+
+
+# ------------------------------------------------------------------ arithmetic
+
+def weight_bytes(m, n, r):
+    return m * n // 2 + 4 * (m // 128) * n + m * r // 2 + 4 * (m // 128) * r + 2 * r * n
+
+
+def act_bytes(b, m, n):
+    return b * m // 2 + 4 * b * (m // 128) + 2 * b * n
+
+
+def int8_ops(b, m, n, r):
+    return 2 * b * m * n + 2 * b * m * r
+
+
+def bf16_flops(b, n, r):
+    return 2 * b * r * n
+
+
+def describe(name):
+    import synth
+    wname, b = WORKLOADS[name]
+    wl = synth.WORKLOADS[wname]
+    return wl, b
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(
+            d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("twq_gemm_sm100.cu", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "rank_residual_w4a4_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary, or None
+    if the summary has no line for this workload or the kernel source changed since."""
+    p = os.path.join(ROOT, "profiles", "fused_kernel_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = kernel_source_hash()
+    with open(p) as fh:
+        for line in fh:
+            parts = line.split()
+            if len(parts) >= 3 and parts[0] == workload and not line.startswith("#"):
+                if parts[2] == want:
+                    return int(parts[1])
+    return None
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the benchmark runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self):
+        return time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvidia-smi unavailable"}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons, power = [], [], set(), []
+        for ts, line in self.lines:
+            if not (t0 - 0.15 <= ts <= t1 + 0.15):
+                continue
+            p = [v.strip() for v in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+                power.append(float(p[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "power_w_max": max(power), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value, world, device):
+    """Max of a float over ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- GPU arm
+
+class Problem:
+    """Device-resident inputs, rotating weight copies and outputs of one workload."""
+
+    def __init__(self, name, device, seed=0, copies=None):
+        import torch
+        import synth
+        from rank_residual_w4a4_b200 import twq
+        self.name = name
+        wl, b = describe(name)
+        self.b, self.m, self.n, self.r = b, wl.m, wl.n, wl.r
+        self.device = device
+        x = synth.make_x(wl, b=b, seed=seed)
+        R, L1, L2 = synth.make_weights(wl, seed=seed)
+        bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        self.x_host = x
+        wb = weight_bytes(self.m, self.n, self.r)
+        if copies is None:
+            copies = max(2, min(32, math.ceil(2 * L2_BYTES / wb)))
+        self.copies = copies
+        w0 = twq.pack_weights(bf(R), bf(L1), bf(L2))
+        self.weights = [w0] + [twq.Weights(w0.m, w0.n, w0.r, w0.rq.clone(), w0.sr.clone(),
+                                           w0.l1q.clone(), w0.sl1.clone(), w0.l2t.clone())
+                               for _ in range(copies - 1)]
+        xd = bf(x)
+        self.x = [xd] + [xd.clone() for _ in range(copies - 1)]
+        self.xq = [torch.empty((b, self.m // 2), dtype=torch.uint8, device=device)
+                   for _ in range(copies)]
+        self.sx = [torch.empty((b, self.m // 128), dtype=torch.float32, device=device)
+                   for _ in range(copies)]
+        self.y = [torch.empty((b, self.n), dtype=torch.bfloat16, device=device) for _ in range(copies)]
+        del R, L1, L2
+
+    def step(self, i, fused=True, ev=None):
+        from rank_residual_w4a4_b200 import twq
+        c = i % self.copies
+        twq.quantize_act(self.x[c], self.xq[c], self.sx[c])
+        if ev is not None:
+            ev[0].record()
+        if fused:
+            twq.fused_linear(self.xq[c], self.sx[c], self.weights[c], self.y[c])
+        if ev is not None:
+            ev[1].record()
+
+
+def capture(fn, count):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        for i in range(count):
+            fn(i)
+    return g
+
+
+def time_graph(g, world, device):
+    import torch
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return s.elapsed_time(e) / 1e3  # seconds
+
+
+def kernel_only_time(prob, fn, steps, reps=1):
+    """Average seconds per launch of `fn(i)` captured back-to-back in a graph."""
+    import torch
+    g = capture(fn, steps)
+    g.replay()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / 1e3 / (steps * reps)
+
+
+def roofline_entry(name, t_kernel, peaks, traffic):
+    wl, b = describe(name)
+    hbm, bf16, bf16_sus, src = peaks
+    m, n, r = wl.m, wl.n, wl.r
+    if b <= 64:  # decode shapes: HBM-bound
+        alg = weight_bytes(m, n, r) + act_bytes(b, m, n)
+        ach = alg / t_kernel / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach / hbm, 4), "traffic": traffic,
+                "peak_source": "%s copy bandwidth" % src, "algorithmic_bytes": alg}
+    ops = int8_ops(b, m, n, r) + bf16_flops(b, n, r)
+    ach = ops / t_kernel / 1e12
+    peak = bf16 * INT8_PER_BF16
+    return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
+            "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": traffic,
+            "peak_source": "%s bf16 burst x %g (nominal int8/bf16 dense ratio)" % (src, INT8_PER_BF16),
+            "algorithmic_ops": ops}
+
+
+def run_gpu(args):
+    import torch
+    world, rank, local = dist_setup()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    from rank_residual_w4a4_b200 import _build, twq
+    _build.build()
+    twq.load()
+    peaks = load_peaks()
+    name = args.workload
+    prob = Problem(name, device)
+    K, W = args.steps, args.warmup
+    wl, b = describe(name)
+
+    # warm-up (eager once, then the warm-up graph), clock sampling from here on
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    prob.step(0)
+    torch.cuda.synchronize()
+    gw = capture(prob.step, W)
+    # sampled per-launch events on the launching stream, every 4th step
+    evs = {}
+
+    def timed_step(i):
+        ev = None
+        if i % 4 == 0:
+            ev = (torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True))
+            evs[i] = ev
+        prob.step(i, ev=ev)
+
+    gk = capture(timed_step, K)
+    t_load0 = time.time()
+    # keep the GPU busy ~1 s so the clock samples see it under load
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        gw.replay()
+        torch.cuda.synchronize()
+    elapsed = time_graph(gk, world, device)
+    t_load1 = time.time()
+    elapsed = max_over_ranks(elapsed, world, device)
+    fused_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in sorted(evs)]
+    t_fused = float(np.mean(fused_ms)) / 1e3
+    st = twq.device_status()
+    if st != 0:
+        raise RuntimeError("device wait timed out at site %d" % st)
+
+    # end to end through the public binding, host buffers, copies inside the timed region
+    e2e = run_e2e(prob, K, W, world, device)
+    clocks.stop()
+    clk = clocks.summary(t_load0, t_load1)
+
+    tokens = b * world * K
+    value = tokens / elapsed
+    ops = int8_ops(b, wl.m, wl.n, wl.r) + bf16_flops(b, wl.n, wl.r)
+    line = {
+        "metric": "fused W4A4+low-rank linear: effective TOPS & tokens/s; % of HBM / INT8 roofline",
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(elapsed / K * 1e3, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4 codes -> int8 MMA (s32 acc) + fp32 scales; bf16 stage 2 and output",
+        "data": "synthetic (seeded generator; no dataset or trained weights)",
+        "config": {"workload": "%s: b=%d m=%d n=%d r=%d, group 128" % (name, b, wl.m, wl.n, wl.r),
+                   "b": b, "m": wl.m, "n": wl.n, "r": wl.r, "parallelism": "replicas x%d" % world,
+                   "step": "twq_quantize_act + twq_fused_linear",
+                   "l2": "weights rotate over %d copies (%.0f MB > 2x L2)" % (
+                       prob.copies, prob.copies * weight_bytes(wl.m, wl.n, wl.r) / 1e6),
+                   "launch": "CUDA graph of the K timed steps"},
+        "effective_tops": round(ops * world * K / elapsed / 1e12, 3),
+        "fused_kernel_us": round(t_fused * 1e6, 3),
+        "roofline": roofline_entry(name, t_fused, peaks, profiled_traffic(name)),
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(name, seconds=args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.no_sweep:
+        line["sweep"] = sweep(args, device, peaks)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del gk, gw
+        dist.destroy_process_group()
+
+
+def run_e2e(prob, K, W, world, device):
+    """Same metric through the Python binding with host buffers: per step an H2D copy of
+    X from pinned memory, quantize + fused layer, and a D2H copy of Y."""
+    import torch
+    from rank_residual_w4a4_b200 import twq
+    xh = torch.from_numpy(prob.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((prob.b, prob.n), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(prob.x[0])
+
+    def one(i):
+        c = i % prob.copies
+        xd.copy_(xh, non_blocking=True)
+        xq, sx = twq.quantize_act(xd, prob.xq[c], prob.sx[c])
+        y = twq.fused_linear(xq, sx, prob.weights[c], prob.y[c])
+        yh.copy_(y, non_blocking=True)
+
+    for i in range(W):
+        one(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(K):
+        one(i)
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    t = max_over_ranks(s.elapsed_time(e) / 1e3, world, device)
+    return {"value": round(prob.b * world * K / t, 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": prob.b * prob.m * 2, "d2h_bytes_per_step": prob.b * prob.n * 2,
+            "path": "python binding, eager launches"}
+
+
+def sweep(args, device, peaks):
+    """Kernel-level numbers of the other workloads: fused, w4a4_only and unfused."""
+    import torch
+    from rank_residual_w4a4_b200 import twq
+    out = []
+    names = [n for n in (args.sweep.split(",") if args.sweep else SWEEP) if n != args.workload]
+    for name in names:
+        prob = Problem(name, device)
+        wl, b = describe(name)
+        steps = 64 if b <= 64 else 8
+        ws = torch.empty(twq.unfused_workspace_bytes(b, wl.n, wl.r), dtype=torch.uint8, device=device)
+        res = {"workload": name, "b": b, "m": wl.m, "n": wl.n, "r": wl.r}
+
+        def fused(i):
+            c = i % prob.copies
+            twq.fused_linear(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c])
+
+        def w4(i):
+            c = i % prob.copies
+            twq.w4a4_only(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c])
+
+        def unf(i):
+            c = i % prob.copies
+            twq.unfused_linear(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c], ws)
+
+        def quant(i):
+            c = i % prob.copies
+            twq.quantize_act(prob.x[c], prob.xq[c], prob.sx[c])
+
+        for i in range(prob.copies):
+            quant(i)
+        torch.cuda.synchronize()
+        t_f = kernel_only_time(prob, fused, steps, reps=3)
+        t_w = kernel_only_time(prob, w4, steps, reps=3)
+        t_u = kernel_only_time(prob, unf, steps, reps=3)
+        t_q = kernel_only_time(prob, quant, steps, reps=3)
+        ops = int8_ops(b, wl.m, wl.n, wl.r) + bf16_flops(b, wl.n, wl.r)
+        res.update({
+            "fused_us": round(t_f * 1e6, 2), "w4a4_only_us": round(t_w * 1e6, 2),
+            "unfused_us": round(t_u * 1e6, 2), "quantize_us": round(t_q * 1e6, 2),
+            "fused_tops": round(ops / t_f / 1e12, 2), "tokens_per_s": round(b / (t_f + t_q), 1),
+            "lowrank_overhead": round(t_f / t_w - 1.0, 4), "fusion_speedup": round(t_u / t_f, 3),
+            "roofline": roofline_entry(name, t_f, peaks, profiled_traffic(name)),
+            "timing": "graph of back-to-back launches, weights rotating over %d copies" % prob.copies,
+        })
+        out.append(res)
+        del prob, ws
+        torch.cuda.empty_cache()
+    st = twq.device_status()
+    if st != 0:
+        raise RuntimeError("device wait timed out at site %d" % st)
+    return out
+
+
+# ------------------------------------------------------------- CPU oracle arm
+
+class OracleProblem:
+    """The oracle on host cores: quantize a sample of rows of X and run the layer for them."""
+
+    def __init__(self, name, seed=0):
+        import oracle
+        import synth
+        wl, b = describe(name)
+        self.b, self.m, self.n, self.r = b, wl.m, wl.n, wl.r
+        self.x = synth.make_x(wl, b=b, seed=seed)
+        R, L1, L2 = synth.make_weights(wl, seed=seed)
+        self.qr, self.sr = oracle.quantize_cols(R)
+        self.ql1, self.sl1 = oracle.quantize_cols(L1)
+        self.L2 = L2
+
+    def rows(self, rows):
+        import oracle
+        xr = self.x[rows]
+        qx, sx = oracle.quantize_rows(xr)
+        oracle.linear(qx, sx, self.qr, self.sr, self.ql1, self.sl1, self.L2, mode=oracle.FUSED)
+
+
+def oracle_rows_parallel(op, row_lists):
+    threads = [threading.Thread(target=op.rows, args=(rl,)) for rl in row_lists]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+
+
+def cpu_baseline(name, seconds=10.0):
+    op = OracleProblem(name)
+    cores = os.cpu_count() or 1
+    # calibrate on one row per core
+    t0 = time.time()
+    oracle_rows_parallel(op, [np.array([i % op.b]) for i in range(cores)])
+    per_round = max(time.time() - t0, 1e-6)
+    rounds = max(1, int(seconds / per_round))
+    rows_per_thread = rounds
+    lists = [np.arange(i * rows_per_thread, (i + 1) * rows_per_thread) % op.b for i in range(cores)]
+    t0 = time.time()
+    oracle_rows_parallel(op, lists)
+    t = time.time() - t0
+    nrows = rows_per_thread * cores
+    return {"value": round(nrows / t, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "%d rows of the %s workload (cycled over its %d tokens), %d threads each "
+                      "running the single-threaded oracle on its own rows; weights quantized "
+                      "outside the timing" % (nrows, name, op.b, cores)}
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    name = args.workload
+    op = OracleProblem(name)
+    cores = os.cpu_count() or 1
+    rows_per_step = max(cores, min(op.b, 16))
+    rows_per_step = (rows_per_step // cores) * cores
+    lists_for = lambda i: [np.arange(rows_per_step // cores) + (i * rows_per_step + c * (rows_per_step // cores))
+                           for c in range(cores)]
+    for i in range(args.warmup):
+        oracle_rows_parallel(op, [l % op.b for l in lists_for(i)])
+    t0 = time.time()
+    for i in range(args.steps):
+        oracle_rows_parallel(op, [l % op.b for l in lists_for(i)])
+    t = time.time() - t0
+    wl, b = describe(name)
+    value = rows_per_step * args.steps / t
+    line = {
+        "metric": "fused W4A4+low-rank linear: effective TOPS & tokens/s; % of HBM / INT8 roofline",
+        "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8 codes, int64 / fp64 accumulation (CPU oracle)",
+        "data": "synthetic (seeded generator; no dataset or trained weights)",
+        "config": {"workload": "%s: b=%d m=%d n=%d r=%d, group 128" % (name, b, wl.m, wl.n, wl.r),
+                   "b": b, "m": wl.m, "n": wl.n, "r": wl.r, "parallelism": "host threads"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": "each step: %d rows of the %s workload over %d threads" % (
+                             rows_per_step, name, cores)},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["twq", "reference"], default="twq")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--sweep", default="", help="comma-separated workloads for the sweep")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

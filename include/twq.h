@@ -1,0 +1,171 @@
+/*
+ * twq.h -- C ABI of the B200 (sm_100a) fused dual-component W4A4 + low-rank
+ * linear layer of TwinQuant ("TwinQuant: Learnable Subspace Decomposition for
+ * 4-Bit LLM Quantization", ICML'26).
+ *
+ * The layer (TwinQuant §2, Eq. (3), with the learned transforms of §4.1 folded
+ * into the factors offline):
+ *
+ *     Y = Q(X) Q(R) + bf16( Q(X) Q(L1) ) L2      X: b x m,  W = L1 L2 + R: m x n
+ *
+ *   Q        symmetric 4-bit quantizer of Eq. (1): codes round(v / s) with
+ *            s = max|v| / 7 (q_max = 2^(4-1) - 1), per group of 128 elements
+ *            along the reduction dimension m (§5.1: group size 128 for weights
+ *            and activations). Rounding is half to even; v / s is a correctly
+ *            rounded float32 division; an all-zero group has s = 0, codes 0.
+ *   stage 1  H = Q(X) Q(L1), b x r, exact int32 per group, scaled in fp32 per
+ *            group (Eq. (2) applied group by group).
+ *   stage 2  H is rounded to BF16 and multiplied by L2 (BF16, unquantized) with
+ *            fp32 accumulation. H never leaves the chip (§4.3: the first
+ *            low-rank GEMM's result is kept on chip and fed to the second).
+ *   epilogue Y = bf16_rne(Y_res + Y_lr), one store (§4.3: a single epilogue
+ *            merges both components).
+ *
+ * Memory: every pointer is a DEVICE pointer owned by the caller; the library
+ * never allocates, frees or synchronizes (except twq_device_status). Every
+ * call is asynchronous on `stream`; inputs must stay live until the stream
+ * reaches the call. All base pointers must be 16-byte aligned.
+ *
+ * Errors: arguments are validated on the host before anything is launched; a
+ * failing check returns a status and launches nothing. A launch failure is
+ * reported as TWQ_ERR_CUDA. Kernels never trap: every wait inside a kernel is
+ * bounded, and a wait that runs out records a code that twq_device_status
+ * returns.
+ *
+ * Formats ("K-major" = the reduction index m is contiguous):
+ *   codes    two's-complement nibbles in [-7, 7], element 2p in the low nibble
+ *            of byte p, element 2p+1 in the high nibble.
+ *   xq, sx   b x (m/2) bytes, row-major; b x (m/128) fp32 scales, row-major.
+ *   rq, sr   n x (m/2) bytes (column j of R, K-major); (m/128) x n fp32.
+ *   l1q, sl1 r x (m/2) bytes (column c of L1, K-major); (m/128) x r fp32.
+ *   l2t      n x r BF16: L2 transposed (K-major for stage 2).
+ *   y        b x n BF16, row-major.
+ * Shapes: m % 128 == 0; n % 128 == 0; r == 0 or (r % 16 == 0 and r <= 256);
+ *   b >= 0 (b == 0 is a no-op).
+ */
+#ifndef TWQ_H_
+#define TWQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TWQ_API __attribute__((visibility("default")))
+#else
+#define TWQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream (NULL = the legacy default stream). */
+typedef struct CUstream_st* twq_stream_t;
+
+typedef enum {
+  TWQ_OK = 0,
+  TWQ_ERR_INVALID_ARG = 1,     /* null pointer, bad shape or size */
+  TWQ_ERR_UNSUPPORTED = 2,     /* valid but outside this build's limits (e.g. r > 256) */
+  TWQ_ERR_MISALIGNED = 3,      /* a pointer or stride breaks the 16-byte rule */
+  TWQ_ERR_CUDA = 4,            /* a CUDA runtime/driver call or launch failed */
+  TWQ_ERR_NOT_IMPLEMENTED = 5,
+  TWQ_ERR_DEVICE = 6           /* a kernel's bounded wait ran out (twq_device_status) */
+} twq_status;
+
+/* Packed weights of one layer (all device pointers, caller-allocated). */
+typedef struct {
+  int64_t m, n, r;
+  uint8_t* rq;   /* n x m/2 */
+  float* sr;     /* m/128 x n */
+  uint8_t* l1q;  /* r x m/2      (may be NULL iff r == 0) */
+  float* sl1;    /* m/128 x r    (may be NULL iff r == 0) */
+  uint16_t* l2t; /* n x r BF16   (may be NULL iff r == 0) */
+} twq_weights;
+
+/* Library version as 10000*major + 100*minor + patch. */
+TWQ_API int twq_version(void);
+
+/* Human-readable name of a status code (static string). */
+TWQ_API const char* twq_status_string(twq_status s);
+
+/*
+ * Byte sizes of the five packed-weight buffers {rq, sr, l1q, sl1, l2t} for an
+ * m x n layer of rank r (TwinQuant §3, Observation 2: the low-rank part adds
+ * r(m + n) parameters; here L1 is 4-bit with per-group scales, L2 is BF16).
+ * Host only; returns TWQ_ERR_INVALID_ARG on a bad shape.
+ */
+TWQ_API twq_status twq_weights_sizes(int64_t m, int64_t n, int64_t r, size_t bytes_out[5]);
+
+/* Byte sizes of {xq, sx} for b tokens of width m. Host only. */
+TWQ_API twq_status twq_act_sizes(int64_t b, int64_t m, size_t bytes_out[2]);
+
+/*
+ * Online activation quantizer (TwinQuant Eq. (1) per token and group of 128;
+ * §4.3: the activation is quantized once and reused by the residual GEMM and
+ * the first low-rank GEMM).
+ *   x    b x m BF16 with row stride ldx elements (ldx >= m, ldx % 8 == 0)
+ *   xq   b x m/2 bytes (output), sx b x m/128 fp32 (output)
+ * Bit-exact with the definition above. X must be finite.
+ */
+TWQ_API twq_status twq_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
+                            float* sx, twq_stream_t stream);
+
+/*
+ * Offline weight packing (TwinQuant §4.1: the transformed factors U', V', R'
+ * are prepared offline; Eq. (1) per output column and group of 128 along m).
+ *   R   m x n BF16 row-major;  L1 m x r BF16 row-major;  L2 r x n BF16 row-major
+ *   out buffers and shape {m, n, r} in *w (sizes from twq_weights_sizes).
+ * R and L1 are quantized (bit-exact); L2 is transposed into l2t unchanged.
+ * L1 and L2 may be NULL iff w->r == 0.
+ */
+TWQ_API twq_status twq_pack_weights(const uint16_t* R, const uint16_t* L1, const uint16_t* L2,
+                            const twq_weights* w, twq_stream_t stream);
+
+/*
+ * The fused dual-component layer (TwinQuant §4.3, Fig. 4): one persistent
+ * kernel that runs the residual GEMM Q(X)Q(R) and the low-rank stage 1
+ * Q(X)Q(L1) on 5th-generation tensor cores (int8 operands unpacked from the
+ * 4-bit codes in shared memory, exact int32 accumulation per group in tensor
+ * memory, fp32 scaling per group), keeps H on chip, rounds it to BF16, runs
+ * stage 2 against L2, and writes Y once.
+ *   xq, sx  from twq_quantize_act;  w  from twq_pack_weights;  y  b x n BF16 (output)
+ * w->r == 0 gives exactly the twq_w4a4_only result.
+ */
+TWQ_API twq_status twq_fused_linear(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                            uint16_t* y, twq_stream_t stream);
+
+/* Residual component only: Y = bf16(Q(X) Q(R)) (TwinQuant Eq. (2)); ignores l1q/sl1/l2t. */
+TWQ_API twq_status twq_w4a4_only(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                         uint16_t* y, twq_stream_t stream);
+
+/* Low-rank component only: Y = bf16(bf16(Q(X) Q(L1)) L2); ignores rq/sr. Needs r > 0. */
+TWQ_API twq_status twq_lowrank_only(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                            uint16_t* y, twq_stream_t stream);
+
+/*
+ * Unfused comparator (the naive schedule that TwinQuant §4.3 describes and
+ * rejects): four launches -- residual GEMM to fp32 Y_res in HBM, stage 1 to
+ * BF16 H in HBM, stage 2 to fp32 Y_lr in HBM, then Y = bf16(Y_res + Y_lr).
+ * Same arithmetic as twq_fused_linear, so the result is bitwise identical.
+ * workspace: device buffer of twq_unfused_workspace_bytes(b, n, r) bytes.
+ */
+TWQ_API size_t twq_unfused_workspace_bytes(int64_t b, int64_t n, int64_t r);
+TWQ_API twq_status twq_unfused_linear(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                              uint16_t* y, void* workspace, size_t workspace_bytes,
+                              twq_stream_t stream);
+
+/*
+ * Reads and clears the device-side status word (SYNCHRONIZES the device).
+ * *code = 0 if no kernel's bounded wait has run out since the last call, else
+ * a site code (which wait gave up). Returns TWQ_ERR_DEVICE if *code != 0.
+ */
+TWQ_API twq_status twq_device_status(int* code);
+
+/* Number of kernels each entry point launches (for launch accounting). */
+TWQ_API int twq_launches_per_call(const char* entry_point);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TWQ_H_ */

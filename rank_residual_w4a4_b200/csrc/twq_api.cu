@@ -1,0 +1,197 @@
+// C ABI of the library (include/twq.h): argument validation on the host, then
+// stream-ordered launches. No entry point allocates device memory.
+#include <string.h>
+
+#include "twq_internal.h"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+twq_status shape_ok(int64_t m, int64_t n, int64_t r) {
+  if (m <= 0 || n <= 0 || r < 0) return TWQ_ERR_INVALID_ARG;
+  if (m % 128 || n % 128) return TWQ_ERR_INVALID_ARG;
+  if (r % 16) return TWQ_ERR_INVALID_ARG;
+  if (r > 256) return TWQ_ERR_UNSUPPORTED;
+  // TMA coordinates and element offsets are 32-bit in the kernels.
+  if (m > (int64_t(1) << 24) || n > (int64_t(1) << 24)) return TWQ_ERR_UNSUPPORTED;
+  return TWQ_OK;
+}
+
+twq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TWQ_OK : TWQ_ERR_CUDA; }
+
+// Checks shared by the three layer entry points. `need_res` / `need_lr` say
+// which weight buffers the call reads.
+twq_status check_layer(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                       const void* y, bool need_res, bool need_lr) {
+  if (!w) return TWQ_ERR_INVALID_ARG;
+  twq_status s = shape_ok(w->m, w->n, w->r);
+  if (s != TWQ_OK) return s;
+  if (b < 0) return TWQ_ERR_INVALID_ARG;
+  if (b > (int64_t(1) << 30)) return TWQ_ERR_UNSUPPORTED;
+  if (b == 0) return TWQ_OK;
+  if (!xq || !sx || !y) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(sx) || !aligned16(y)) return TWQ_ERR_MISALIGNED;
+  if (need_res) {
+    if (!w->rq || !w->sr) return TWQ_ERR_INVALID_ARG;
+    if (!aligned16(w->rq) || !aligned16(w->sr)) return TWQ_ERR_MISALIGNED;
+  }
+  if (need_lr) {
+    if (w->r == 0) return TWQ_ERR_INVALID_ARG;
+    if (!w->l1q || !w->sl1 || !w->l2t) return TWQ_ERR_INVALID_ARG;
+    if (!aligned16(w->l1q) || !aligned16(w->sl1) || !aligned16(w->l2t)) return TWQ_ERR_MISALIGNED;
+  }
+  return TWQ_OK;
+}
+
+twq_status run(int mode, const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+               void* out, const uint16_t* h, twq_stream_t stream) {
+  twq::GemmCall c{mode, xq, sx, b, w, out, h};
+  return from_cuda(twq::launch_gemm(c, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+}  // namespace
+
+extern "C" {
+
+int twq_version(void) { return kVersion; }
+
+const char* twq_status_string(twq_status s) {
+  switch (s) {
+    case TWQ_OK: return "ok";
+    case TWQ_ERR_INVALID_ARG: return "invalid argument";
+    case TWQ_ERR_UNSUPPORTED: return "unsupported shape";
+    case TWQ_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case TWQ_ERR_CUDA: return "CUDA error";
+    case TWQ_ERR_NOT_IMPLEMENTED: return "not implemented";
+    case TWQ_ERR_DEVICE: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+twq_status twq_weights_sizes(int64_t m, int64_t n, int64_t r, size_t bytes_out[5]) {
+  if (!bytes_out) return TWQ_ERR_INVALID_ARG;
+  twq_status s = shape_ok(m, n, r);
+  if (s != TWQ_OK) return s;
+  const int64_t G = m / 128;
+  bytes_out[0] = static_cast<size_t>(n * (m / 2));
+  bytes_out[1] = static_cast<size_t>(G * n * 4);
+  bytes_out[2] = static_cast<size_t>(r * (m / 2));
+  bytes_out[3] = static_cast<size_t>(G * r * 4);
+  bytes_out[4] = static_cast<size_t>(n * r * 2);
+  return TWQ_OK;
+}
+
+twq_status twq_act_sizes(int64_t b, int64_t m, size_t bytes_out[2]) {
+  if (!bytes_out || b < 0 || m <= 0 || m % 128) return TWQ_ERR_INVALID_ARG;
+  bytes_out[0] = static_cast<size_t>(b * (m / 2));
+  bytes_out[1] = static_cast<size_t>(b * (m / 128) * 4);
+  return TWQ_OK;
+}
+
+twq_status twq_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
+                            float* sx, twq_stream_t stream) {
+  if (b < 0 || m <= 0 || m % 128 || ldx < m) return TWQ_ERR_INVALID_ARG;
+  if (m > (int64_t(1) << 24) || b > (int64_t(1) << 30)) return TWQ_ERR_UNSUPPORTED;
+  if (b == 0) return TWQ_OK;
+  if (!x || !xq || !sx) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(sx) || ldx % 8) return TWQ_ERR_MISALIGNED;
+  return from_cuda(twq::launch_quantize_act(x, b, m, ldx, xq, sx,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+twq_status twq_pack_weights(const uint16_t* R, const uint16_t* L1, const uint16_t* L2,
+                            const twq_weights* w, twq_stream_t stream) {
+  if (!w) return TWQ_ERR_INVALID_ARG;
+  twq_status s = shape_ok(w->m, w->n, w->r);
+  if (s != TWQ_OK) return s;
+  if (!R || !w->rq || !w->sr) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(R) || !aligned16(w->rq) || !aligned16(w->sr)) return TWQ_ERR_MISALIGNED;
+  if (w->r > 0) {
+    if (!L1 || !L2 || !w->l1q || !w->sl1 || !w->l2t) return TWQ_ERR_INVALID_ARG;
+    if (!aligned16(L1) || !aligned16(L2) || !aligned16(w->l1q) || !aligned16(w->sl1) ||
+        !aligned16(w->l2t))
+      return TWQ_ERR_MISALIGNED;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = twq::launch_pack_cols(R, w->m, w->n, w->rq, w->sr, st);
+  if (e == cudaSuccess && w->r > 0) e = twq::launch_pack_cols(L1, w->m, w->r, w->l1q, w->sl1, st);
+  if (e == cudaSuccess && w->r > 0) e = twq::launch_transpose_bf16(L2, w->r, w->n, w->l2t, st);
+  return from_cuda(e);
+}
+
+twq_status twq_fused_linear(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                            uint16_t* y, twq_stream_t stream) {
+  const bool lr = w && w->r > 0;
+  twq_status s = check_layer(xq, sx, b, w, y, true, lr);
+  if (s != TWQ_OK || b == 0) return s;
+  return run(lr ? twq::kModeFused : twq::kModeW4A4, xq, sx, b, w, y, nullptr, stream);
+}
+
+twq_status twq_w4a4_only(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                         uint16_t* y, twq_stream_t stream) {
+  twq_status s = check_layer(xq, sx, b, w, y, true, false);
+  if (s != TWQ_OK || b == 0) return s;
+  return run(twq::kModeW4A4, xq, sx, b, w, y, nullptr, stream);
+}
+
+twq_status twq_lowrank_only(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                            uint16_t* y, twq_stream_t stream) {
+  twq_status s = check_layer(xq, sx, b, w, y, false, true);
+  if (s != TWQ_OK || b == 0) return s;
+  return run(twq::kModeLowRank, xq, sx, b, w, y, nullptr, stream);
+}
+
+size_t twq_unfused_workspace_bytes(int64_t b, int64_t n, int64_t r) {
+  if (b <= 0 || n <= 0 || r < 0) return 0;
+  // Y_res fp32 (b x n) | Y_lr fp32 (b x n) | H bf16 (b x r), each 256-byte aligned
+  auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
+  return up(size_t(b) * n * 4) * 2 + up(size_t(b) * r * 2);
+}
+
+twq_status twq_unfused_linear(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                              uint16_t* y, void* workspace, size_t workspace_bytes,
+                              twq_stream_t stream) {
+  const bool lr = w && w->r > 0;
+  twq_status s = check_layer(xq, sx, b, w, y, true, lr);
+  if (s != TWQ_OK || b == 0) return s;
+  if (!workspace) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return TWQ_ERR_MISALIGNED;
+  if (workspace_bytes < twq_unfused_workspace_bytes(b, w->n, w->r)) return TWQ_ERR_INVALID_ARG;
+  auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* yres = reinterpret_cast<float*>(ws);
+  float* ylr = reinterpret_cast<float*>(ws + up(size_t(b) * w->n * 4));
+  uint16_t* h = reinterpret_cast<uint16_t*>(ws + 2 * up(size_t(b) * w->n * 4));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!lr) return run(twq::kModeW4A4, xq, sx, b, w, y, nullptr, stream);
+  s = run(twq::kModeResF32, xq, sx, b, w, yres, nullptr, stream);
+  if (s == TWQ_OK) s = run(twq::kModeHOnly, xq, sx, b, w, h, nullptr, stream);
+  if (s == TWQ_OK) s = run(twq::kModeS2F32, xq, sx, b, w, ylr, h, stream);
+  if (s == TWQ_OK) s = from_cuda(twq::launch_add_cast(yres, ylr, b * w->n, y, st));
+  return s;
+}
+
+twq_status twq_device_status(int* code) {
+  if (!code) return TWQ_ERR_INVALID_ARG;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return TWQ_ERR_CUDA;
+  e = twq::read_and_clear_device_status(code);
+  if (e != cudaSuccess) return TWQ_ERR_CUDA;
+  return *code ? TWQ_ERR_DEVICE : TWQ_OK;
+}
+
+int twq_launches_per_call(const char* ep) {
+  if (!ep) return -1;
+  if (!strcmp(ep, "twq_quantize_act")) return 1;
+  if (!strcmp(ep, "twq_pack_weights")) return 3;
+  if (!strcmp(ep, "twq_fused_linear") || !strcmp(ep, "twq_w4a4_only") ||
+      !strcmp(ep, "twq_lowrank_only"))
+    return 1;
+  if (!strcmp(ep, "twq_unfused_linear")) return 4;
+  return -1;
+}
+
+}  // extern "C"

@@ -1,0 +1,783 @@
+// Tensor-core kernel of the dual-component W4A4 + low-rank linear layer for
+// sm_100a (TwinQuant, "Learnable Subspace Decomposition for 4-Bit LLM
+// Quantization", §4.3 "Dual-Component Kernel Design" and Fig. 4).
+//
+// One persistent CTA per SM walks a contiguous run of 128 x BN output tiles
+// (row-block major). For each tile:
+//   * stage 1 (only when the row block changes): H = Q(X) Q(L1) over all
+//     m/128 groups, int32 per group in tensor memory, scaled by
+//     sx[i,g] * sl1[g,c] in fp32 and summed in registers; then H -> BF16 into a
+//     shared-memory operand tile that later tiles of the same row block reuse
+//     (H never goes to HBM);
+//   * residual: Y_res = sum_g sx[i,g] sr[g,j] (Q(X)_g Q(R)_g), same scheme;
+//   * stage 2: Y_lr = bf16(H) L2 with kind::f16 MMAs (fp32 accumulation);
+//   * one epilogue: Y = bf16(Y_res + Y_lr), a single store.
+//
+// Warp roles (512 threads):
+//   warp 0        TMA producer: packed 4-bit code tiles of X and R / L1, BF16
+//                 tiles of L2^T, and the per-group weight scales;
+//   warp 1        tcgen05.mma issuer (one thread) and TMEM owner;
+//   warps 4-7     unpack: 4-bit codes -> int8 in the UMMA 128-byte-swizzle
+//                 K-major layout (each byte holds 16*q; the MMA result is 256x
+//                 the integer dot product and is rescaled exactly by 2^-8);
+//   warps 8-15    drain: per-group tensor-memory loads, fp32 scaling and
+//                 accumulation, H -> BF16, epilogue.
+// Inside every 16-byte chunk the unpack writes the even-index codes first and
+// the odd-index codes second; A and B use the same order, so every product
+// still pairs the same k and the per-group integer sums are unchanged.
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+#include "twq_internal.h"
+
+namespace twq {
+
+__device__ int g_device_status;
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kBM = 128;
+constexpr int kPackedStages = 4;
+constexpr int kUnpackedStages = 2;
+constexpr int kScaleSlots = 4;
+constexpr int kHChunk = 128;  // H columns per stage-1 pass
+constexpr int kMaxRank = 256;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a wait that lasts 2 s is a failure
+
+template <int kMode>
+struct ModeTraits {
+  static constexpr bool res = kMode == kModeFused || kMode == kModeW4A4 || kMode == kModeResF32;
+  static constexpr bool h = kMode == kModeFused || kMode == kModeLowRank || kMode == kModeHOnly;
+  static constexpr bool s2 = kMode == kModeFused || kMode == kModeLowRank || kMode == kModeS2F32;
+  static constexpr bool h_global = kMode == kModeS2F32;
+  static constexpr bool out_f32 = kMode == kModeResF32 || kMode == kModeS2F32;
+  static constexpr bool out_h = kMode == kModeHOnly;
+};
+
+template <int BN>
+struct SmemLayout {
+  static constexpr int kSlotA = 8192;  // 128 rows x 64 packed bytes
+  static constexpr int kSlot = (kSlotA + BN * 64) > BN * 128 ? (kSlotA + BN * 64) : BN * 128;
+  static constexpr int kUA = 16384;   // 128 rows x 128 int8
+  static constexpr int kUB = BN * 128;
+  static constexpr int kUStage = kUA + kUB;
+  static constexpr int kHb = kBM * kMaxRank * 2;  // up to 4 K-chunks of 128 x 64 BF16
+  static constexpr int kScaleSlot = BN * 4;
+  static constexpr int kOffSlots = 0;
+  static constexpr int kOffU = kOffSlots + kPackedStages * kSlot;
+  static constexpr int kOffHb = kOffU + kUnpackedStages * kUStage;
+  static constexpr int kOffScale = kOffHb + kHb;
+  static constexpr int kOffBar = kOffScale + kScaleSlots * kScaleSlot;
+  static constexpr int kNumBars = 2 * kPackedStages + 2 * kUnpackedStages + 4 + 2 * kScaleSlots + 3;
+  static constexpr int kBytes = kOffBar + kNumBars * 8 + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
+  static constexpr int kTmemCols = 2 * BN;      // two accumulator buffers
+  static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+  static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of 2");
+};
+
+struct GemmArgs {
+  const float* sx;
+  const float* sr;
+  const float* sl1;
+  void* out;
+  int64_t b;
+  int m, n, r, G;
+  int row_blocks, col_tiles, num_tiles;
+  int r_pad;  // stage-2 K extent: r rounded up to 64
+  int h_box;  // rows of the L1 TMA box: min(r, 128)
+};
+
+struct Ring {
+  int idx = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++idx == n) {
+      idx = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+__device__ __forceinline__ void record_failure(int site) {
+  atomicCAS(&g_device_status, 0, site);
+}
+
+// Bounded wait on a barrier phase. Returns false if the CTA is aborting or the
+// wait ran out (then it records `site` and raises the abort flag).
+__device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                      int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      record_failure(site);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Offset of 16-byte chunk `c` of row `row` in a K-major 128-byte-swizzle tile.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int c) {
+  return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
+}
+
+// 4-bit codes (rows x 64 bytes, dense) -> int8 (rows x 128 bytes, swizzled), 16*q per byte.
+__device__ __forceinline__ void unpack_rows(const uint8_t* src, uint8_t* dst, int rows, int tid,
+                                            int nthreads) {
+  const int chunks = rows * 8;
+  for (int e = tid; e < chunks; e += nthreads) {
+    const int row = e >> 3;
+    const int c = e & 7;
+    const uint2 w = *reinterpret_cast<const uint2*>(src + row * 64 + c * 8);
+    uint4 o;
+    o.x = (w.x << 4) & 0xF0F0F0F0u;
+    o.y = w.x & 0xF0F0F0F0u;
+    o.z = (w.y << 4) & 0xF0F0F0F0u;
+    o.w = w.y & 0xF0F0F0F0u;
+    *reinterpret_cast<uint4*>(dst + sw128_offset(row, c)) = o;
+  }
+}
+
+__device__ __forceinline__ void copy_smem(const uint8_t* src, uint8_t* dst, int bytes, int tid,
+                                          int nthreads) {
+  for (int off = tid * 16; off < bytes; off += nthreads * 16)
+    *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src + off);
+}
+
+// acc[j] += float(I[j]) * sc[j] * sx for this thread's lane and ncols columns
+// (ncols % 8 == 0, <= 64) of the int32 accumulator at taddr.
+__device__ __forceinline__ void drain_group(float (&acc)[64], uint32_t taddr, int ncols,
+                                            const float* sc, float sx) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t v[32];
+#pragma unroll
+    for (int c = 0; c < 32; c += 8)
+      if (h * 32 + c < ncols) {
+        uint32_t t[8];
+        tmem_ld8(taddr + h * 32 + c, t);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[c + k] = t[k];
+      }
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 32; c += 4)
+      if (h * 32 + c < ncols) {
+        const float4 s4 = *reinterpret_cast<const float4*>(sc + h * 32 + c);
+        acc[h * 32 + c + 0] =
+            fmaf(static_cast<float>(static_cast<int32_t>(v[c + 0])) * s4.x, sx, acc[h * 32 + c + 0]);
+        acc[h * 32 + c + 1] =
+            fmaf(static_cast<float>(static_cast<int32_t>(v[c + 1])) * s4.y, sx, acc[h * 32 + c + 1]);
+        acc[h * 32 + c + 2] =
+            fmaf(static_cast<float>(static_cast<int32_t>(v[c + 2])) * s4.z, sx, acc[h * 32 + c + 2]);
+        acc[h * 32 + c + 3] =
+            fmaf(static_cast<float>(static_cast<int32_t>(v[c + 3])) * s4.w, sx, acc[h * 32 + c + 3]);
+      }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+struct TileInfo {
+  int rb, ct;
+  bool need_h;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, int t, int t_begin, bool has_h) {
+  TileInfo ti;
+  ti.rb = t / a.col_tiles;
+  ti.ct = t % a.col_tiles;
+  ti.need_h = has_h && (t == t_begin || (t - 1) / a.col_tiles != ti.rb);
+  return ti;
+}
+
+template <int kMode, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    twq_gemm_kernel(const __grid_constant__ CUtensorMap tm_xq,
+                    const __grid_constant__ CUtensorMap tm_rq,
+                    const __grid_constant__ CUtensorMap tm_l1q,
+                    const __grid_constant__ CUtensorMap tm_l2t,
+                    const __grid_constant__ CUtensorMap tm_h, const GemmArgs args) {
+  using L = SmemLayout<BN>;
+  using T = ModeTraits<kMode>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_abort;
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* slots = smem + L::kOffSlots;
+  uint8_t* ustg = smem + L::kOffU;
+  uint8_t* hb = smem + L::kOffHb;
+  float* scl = reinterpret_cast<float*>(smem + L::kOffScale);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = full + kPackedStages;
+  uint64_t* ufull = empty + kPackedStages;
+  uint64_t* uempty = ufull + kUnpackedStages;
+  uint64_t* acc_full = uempty + kUnpackedStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* sc_full = acc_empty + 2;
+  uint64_t* sc_empty = sc_full + kScaleSlots;
+  uint64_t* hb_ready = sc_empty + kScaleSlots;
+  uint64_t* hb_free = hb_ready + 1;
+  uint64_t* mma_done = hb_free + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = &s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = args.G;
+  const int HC = T::h ? (args.r + kHChunk - 1) / kHChunk : 0;
+  const int KC = args.r_pad / 64;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPackedStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);
+    }
+    for (int i = 0; i < kUnpackedStages; ++i) {
+      mbar_init(&ufull[i], 4);
+      mbar_init(&uempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 8);
+    }
+    for (int i = 0; i < kScaleSlots; ++i) {
+      mbar_init(&sc_full[i], 1);
+      mbar_init(&sc_empty[i], 8);
+    }
+    mbar_init(hb_ready, T::h_global ? 1 : 8);
+    mbar_init(hb_free, 1);
+    mbar_init(mma_done, 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&tm_xq);
+    if (T::res) tma_prefetch_desc(&tm_rq);
+    if (T::h) tma_prefetch_desc(&tm_l1q);
+    if (T::s2) tma_prefetch_desc(&tm_l2t);
+    if (T::h_global) tma_prefetch_desc(&tm_h);
+  }
+  // Zero the K padding [r, r_pad) of the on-chip H operand (stage 2 reads it).
+  if (T::s2 && !T::h_global) {
+    const int pad_units = (args.r_pad - args.r) / 8;
+    for (int e = threadIdx.x; e < kBM * pad_units; e += kThreads) {
+      const int row = e / pad_units;
+      const int col = args.r + (e % pad_units) * 8;
+      *reinterpret_cast<uint4*>(hb + (col >> 6) * 16384 + sw128_offset(row, (col & 63) >> 3)) =
+          make_uint4(0, 0, 0, 0);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, L::kTmemCols);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int t_begin = static_cast<int>((int64_t)blockIdx.x * args.num_tiles / gridDim.x);
+  const int t_end = static_cast<int>((int64_t)(blockIdx.x + 1) * args.num_tiles / gridDim.x);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      Ring s, q;
+      uint32_t hb_phase = 0;
+      bool hb_pend = false;
+      bool pend[kPackedStages] = {};
+      uint32_t pend_phase[kPackedStages];
+      bool spend[kScaleSlots] = {};
+      uint32_t spend_phase[kScaleSlots];
+      bool ok = true;
+      for (int t = t_begin; t < t_end && ok; ++t) {
+        const TileInfo ti = tile_info(args, t, t_begin, T::h);
+        const int row0 = ti.rb * kBM;
+        const int n0 = ti.ct * BN;
+        if (ti.need_h) {
+          for (int hc = 0; hc < HC && ok; ++hc) {
+            const int nh = min(kHChunk, args.r - hc * kHChunk);
+            for (int g = 0; g < G; ++g) {
+              if (!(ok = wait_bar(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
+                break;
+              uint8_t* slot = slots + s.idx * L::kSlot;
+              mbar_arrive_expect_tx(&full[s.idx], L::kSlotA + args.h_box * 64);
+              tma_load_2d(slot, &tm_xq, &full[s.idx], g * 64, row0);
+              tma_load_2d(slot + L::kSlotA, &tm_l1q, &full[s.idx], g * 64, hc * kHChunk);
+              pend[s.idx] = true;
+              pend_phase[s.idx] = s.phase;
+              s.next(kPackedStages);
+              if (!(ok = wait_bar(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
+                                  kSiteProducerScaleEmpty)))
+                break;
+              mbar_arrive_expect_tx(&sc_full[q.idx], nh * 4);
+              bulk_load(scl + q.idx * BN, args.sl1 + (int64_t)g * args.r + hc * kHChunk, nh * 4,
+                        &sc_full[q.idx]);
+              spend[q.idx] = true;
+              spend_phase[q.idx] = q.phase;
+              q.next(kScaleSlots);
+            }
+          }
+        }
+        if (T::res && ok) {
+          for (int g = 0; g < G; ++g) {
+            if (!(ok = wait_bar(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
+              break;
+            uint8_t* slot = slots + s.idx * L::kSlot;
+            mbar_arrive_expect_tx(&full[s.idx], L::kSlotA + BN * 64);
+            tma_load_2d(slot, &tm_xq, &full[s.idx], g * 64, row0);
+            tma_load_2d(slot + L::kSlotA, &tm_rq, &full[s.idx], g * 64, n0);
+            pend[s.idx] = true;
+            pend_phase[s.idx] = s.phase;
+            s.next(kPackedStages);
+            if (!(ok = wait_bar(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
+                                kSiteProducerScaleEmpty)))
+              break;
+            mbar_arrive_expect_tx(&sc_full[q.idx], BN * 4);
+            bulk_load(scl + q.idx * BN, args.sr + (int64_t)g * args.n + n0, BN * 4,
+                      &sc_full[q.idx]);
+            spend[q.idx] = true;
+            spend_phase[q.idx] = q.phase;
+            q.next(kScaleSlots);
+          }
+        }
+        if (T::s2 && ok) {
+          if (T::h_global) {
+            if (!(ok = wait_bar(hb_free, hb_phase ^ 1u, abort_flag, kSiteProducerHbFree))) break;
+            mbar_arrive_expect_tx(hb_ready, KC * 16384);
+            for (int kc = 0; kc < KC; ++kc)
+              tma_load_2d(hb + kc * 16384, &tm_h, hb_ready, kc * 64, row0);
+            hb_pend = true;
+            hb_phase ^= 1u;
+          }
+          for (int kc = 0; kc < KC; ++kc) {
+            if (!(ok = wait_bar(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
+              break;
+            mbar_arrive_expect_tx(&full[s.idx], BN * 128);
+            tma_load_2d(slots + s.idx * L::kSlot, &tm_l2t, &full[s.idx], kc * 64, n0);
+            pend[s.idx] = true;
+            pend_phase[s.idx] = s.phase;
+            s.next(kPackedStages);
+          }
+        }
+      }
+      if (!ok) {
+        // Aborting: let the copies already issued land before the CTA exits.
+        int dummy = 0;
+        volatile int* never = &dummy;
+        for (int i = 0; i < kPackedStages; ++i)
+          if (pend[i]) wait_bar(&full[i], pend_phase[i], never, kSiteFinal);
+        for (int i = 0; i < kScaleSlots; ++i)
+          if (spend[i]) wait_bar(&sc_full[i], spend_phase[i], never, kSiteFinal);
+        if (T::h_global && hb_pend) wait_bar(hb_ready, hb_phase ^ 1u, never, kSiteFinal);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      Ring u, a;
+      uint32_t hb_phase = 0;
+      bool ok = true;
+      const uint32_t ua0 = smem_u32(ustg);
+      const uint32_t hb0 = smem_u32(hb);
+      for (int t = t_begin; t < t_end && ok; ++t) {
+        const TileInfo ti = tile_info(args, t, t_begin, T::h);
+        if (ti.need_h) {
+          for (int hc = 0; hc < HC && ok; ++hc) {
+            const int nh = min(kHChunk, args.r - hc * kHChunk);
+            const uint32_t idesc = idesc_i8(nh);
+            for (int g = 0; g < G; ++g) {
+              if (!(ok = wait_bar(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
+              if (!(ok = wait_bar(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
+                break;
+              tc_fence_after();
+              const uint32_t d = tmem_base + a.idx * BN;
+              const uint64_t da = smem_desc_sw128(ua0 + u.idx * L::kUStage);
+              const uint64_t db = smem_desc_sw128(ua0 + u.idx * L::kUStage + L::kUA);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) mma_i8(d, da + 2 * k, db + 2 * k, idesc, k > 0);
+              mma_commit(&uempty[u.idx]);
+              mma_commit(&acc_full[a.idx]);
+              u.next(kUnpackedStages);
+              a.next(2);
+            }
+          }
+        }
+        if (T::res && ok) {
+          const uint32_t idesc = idesc_i8(BN);
+          for (int g = 0; g < G; ++g) {
+            if (!(ok = wait_bar(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
+            if (!(ok = wait_bar(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
+              break;
+            tc_fence_after();
+            const uint32_t d = tmem_base + a.idx * BN;
+            const uint64_t da = smem_desc_sw128(ua0 + u.idx * L::kUStage);
+            const uint64_t db = smem_desc_sw128(ua0 + u.idx * L::kUStage + L::kUA);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mma_i8(d, da + 2 * k, db + 2 * k, idesc, k > 0);
+            mma_commit(&uempty[u.idx]);
+            mma_commit(&acc_full[a.idx]);
+            u.next(kUnpackedStages);
+            a.next(2);
+          }
+        }
+        if (T::s2 && ok) {
+          if (ti.need_h || T::h_global) {
+            if (!(ok = wait_bar(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) break;
+            hb_phase ^= 1u;
+          }
+          if (!(ok = wait_bar(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
+            break;
+          const uint32_t idesc = idesc_bf16(BN);
+          const uint32_t d = tmem_base + a.idx * BN;
+          for (int kc = 0; kc < KC; ++kc) {
+            if (!(ok = wait_bar(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
+            tc_fence_after();
+            const uint64_t da = smem_desc_sw128(hb0 + kc * 16384);
+            const uint64_t db = smem_desc_sw128(ua0 + u.idx * L::kUStage + L::kUA);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16(d, da + 2 * k, db + 2 * k, idesc, (kc | k) != 0);
+            mma_commit(&uempty[u.idx]);
+            u.next(kUnpackedStages);
+          }
+          if (!ok) break;
+          mma_commit(&acc_full[a.idx]);
+          if (T::h_global) mma_commit(hb_free);
+          a.next(2);
+        }
+      }
+      // All MMAs issued by this thread are complete before TMEM is released.
+      mma_commit(mma_done);
+      int dummy = 0;
+      wait_bar(mma_done, 0, &dummy, kSiteFinal);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // --------------------------------------------------------------- unpack
+    const int tid = threadIdx.x - 128;
+    Ring s, u;
+    bool ok = true;
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const TileInfo ti = tile_info(args, t, t_begin, T::h);
+      const int n_h = ti.need_h ? HC * G : 0;
+      const int n_res = T::res ? G : 0;
+      const int n_l2 = T::s2 ? KC : 0;
+      for (int step = 0; step < n_h + n_res + n_l2; ++step) {
+        if (!(ok = wait_bar(&full[s.idx], s.phase, abort_flag, kSiteUnpackFull))) break;
+        if (!(ok = wait_bar(&uempty[u.idx], u.phase ^ 1u, abort_flag, kSiteUnpackEmpty))) break;
+        const uint8_t* src = slots + s.idx * L::kSlot;
+        uint8_t* dst = ustg + u.idx * L::kUStage;
+        if (step < n_h + n_res) {
+          int brows = BN;
+          if (step < n_h) {
+            const int hc = step / G;
+            brows = min(kHChunk, args.r - hc * kHChunk);
+          }
+          unpack_rows(src, dst, kBM, tid, 128);
+          unpack_rows(src + L::kSlotA, dst + L::kUA, brows, tid, 128);
+        } else {
+          copy_smem(src, dst + L::kUA, BN * 128, tid, 128);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&ufull[u.idx]);
+          mbar_arrive(&empty[s.idx]);
+        }
+        s.next(kPackedStages);
+        u.next(kUnpackedStages);
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------------------------------------------------------- drain
+    const int dw = warp - 8;
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int half = dw >> 2;      // which half of the tile's columns
+    const int row_in = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    Ring a, q;
+    bool ok = true;
+    float acc[64];
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const TileInfo ti = tile_info(args, t, t_begin, T::h);
+      const int64_t row = static_cast<int64_t>(ti.rb) * kBM + row_in;
+      const bool row_ok = row < args.b;
+      const float* sx_row = args.sx + (row_ok ? row : 0) * G;
+      const int n0 = ti.ct * BN;
+      if (ti.need_h) {
+        for (int hc = 0; hc < HC && ok; ++hc) {
+          const int nh = min(kHChunk, args.r - hc * kHChunk);
+          const int ncols = nh / 2;
+          const int c0 = half * ncols;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+          for (int g = 0; g < G; ++g) {
+            const float sx = row_ok ? __ldg(sx_row + g) : 0.0f;
+            if (!(ok = wait_bar(&acc_full[a.idx], a.phase, abort_flag, kSiteDrainAccFull))) break;
+            tc_fence_after();
+            if (!(ok = wait_bar(&sc_full[q.idx], q.phase, abort_flag, kSiteDrainScaleFull))) break;
+            drain_group(acc, tmem_base + lane_addr + a.idx * BN + c0, ncols, scl + q.idx * BN + c0,
+                        sx);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&acc_empty[a.idx]);
+              mbar_arrive(&sc_empty[q.idx]);
+            }
+            a.next(2);
+            q.next(kScaleSlots);
+          }
+          if (!ok) break;
+          // H chunk complete: 2^-8 undoes the 16x16 code scaling of the unpack.
+#pragma unroll
+          for (int j = 0; j < 64; j += 8) {
+            if (j < ncols) {
+              uint4 o;
+              o.x = pack_bf16x2(acc[j + 0] * 0.00390625f, acc[j + 1] * 0.00390625f);
+              o.y = pack_bf16x2(acc[j + 2] * 0.00390625f, acc[j + 3] * 0.00390625f);
+              o.z = pack_bf16x2(acc[j + 4] * 0.00390625f, acc[j + 5] * 0.00390625f);
+              o.w = pack_bf16x2(acc[j + 6] * 0.00390625f, acc[j + 7] * 0.00390625f);
+              const int col = hc * kHChunk + c0 + j;
+              if (T::out_h) {
+                if (row_ok)
+                  *reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.out) + row * args.r +
+                                            col) = o;
+              } else {
+                *reinterpret_cast<uint4*>(hb + (col >> 6) * 16384 +
+                                          sw128_offset(row_in, (col & 63) >> 3)) = o;
+              }
+            }
+          }
+        }
+        if (!ok) break;
+        if (!T::out_h) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(hb_ready);
+        }
+      }
+      if (T::out_h) continue;
+      const int ncols = BN / 2;
+      const int c0 = half * ncols;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+      if (T::res) {
+        for (int g = 0; g < G; ++g) {
+          const float sx = row_ok ? __ldg(sx_row + g) : 0.0f;
+          if (!(ok = wait_bar(&acc_full[a.idx], a.phase, abort_flag, kSiteDrainAccFull))) break;
+          tc_fence_after();
+          if (!(ok = wait_bar(&sc_full[q.idx], q.phase, abort_flag, kSiteDrainScaleFull))) break;
+          drain_group(acc, tmem_base + lane_addr + a.idx * BN + c0, ncols, scl + q.idx * BN + c0,
+                      sx);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&acc_empty[a.idx]);
+            mbar_arrive(&sc_empty[q.idx]);
+          }
+          a.next(2);
+          q.next(kScaleSlots);
+        }
+        if (!ok) break;
+      }
+      // -------------------------------------------------------- epilogue
+      // 16 columns at a time: stage-2 result from TMEM, plus the residual sum.
+      if (T::s2) {
+        if (!(ok = wait_bar(&acc_full[a.idx], a.phase, abort_flag, kSiteDrainAccFull))) break;
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int j = 0; j < 64; j += 16) {
+        float lr[16];
+        if (T::s2) {
+          uint32_t t0[8], t1[8];
+          tmem_ld8(tmem_base + lane_addr + a.idx * BN + c0 + j, t0);
+          tmem_ld8(tmem_base + lane_addr + a.idx * BN + c0 + j + 8, t1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            lr[k] = __uint_as_float(t0[k]);
+            lr[k + 8] = __uint_as_float(t1[k]);
+          }
+        }
+        if (row_ok) {
+          if (T::out_f32) {
+            float* o = static_cast<float*>(args.out) + row * args.n + n0 + c0 + j;
+#pragma unroll
+            for (int k = 0; k < 16; k += 4) {
+              float4 v;
+              if (T::res)
+                v = make_float4(acc[j + k] * 0.00390625f, acc[j + k + 1] * 0.00390625f,
+                                acc[j + k + 2] * 0.00390625f, acc[j + k + 3] * 0.00390625f);
+              else
+                v = make_float4(lr[k], lr[k + 1], lr[k + 2], lr[k + 3]);
+              *reinterpret_cast<float4*>(o + k) = v;
+            }
+          } else {
+            uint16_t* o = static_cast<uint16_t*>(args.out) + row * args.n + n0 + c0 + j;
+            float y[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              if (T::s2)
+                y[k] = acc[j + k] * 0.00390625f + lr[k];
+              else
+                y[k] = acc[j + k] * 0.00390625f;
+            }
+#pragma unroll
+            for (int k = 0; k < 16; k += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(y[k + 0], y[k + 1]);
+              v.y = pack_bf16x2(y[k + 2], y[k + 3]);
+              v.z = pack_bf16x2(y[k + 4], y[k + 5]);
+              v.w = pack_bf16x2(y[k + 6], y[k + 7]);
+              *reinterpret_cast<uint4*>(o + k) = v;
+            }
+          }
+        }
+      }
+      if (T::s2) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[a.idx]);
+        a.next(2);
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+template <int kMode, int BN>
+cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
+  using L = SmemLayout<BN>;
+  using T = ModeTraits<kMode>;
+  const twq_weights* w = c.w;
+  GemmArgs a{};
+  a.sx = c.sx;
+  a.sr = w->sr;
+  a.sl1 = w->sl1;
+  a.out = c.out;
+  a.b = c.b;
+  a.m = static_cast<int>(w->m);
+  a.n = static_cast<int>(w->n);
+  a.r = static_cast<int>(w->r);
+  a.G = a.m / 128;
+  a.row_blocks = static_cast<int>((c.b + kBM - 1) / kBM);
+  a.col_tiles = T::out_h ? 1 : a.n / BN;
+  a.num_tiles = a.row_blocks * a.col_tiles;
+  a.r_pad = ((a.r + 63) / 64) * 64;
+  a.h_box = a.r < kHChunk ? a.r : kHChunk;
+
+  CUtensorMap m_xq{}, m_rq{}, m_l1q{}, m_l2t{}, m_h{};
+  const uint64_t kb = static_cast<uint64_t>(a.m / 2);
+  bool ok = encode_2d(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, kb, c.b, kb, 64, kBM,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (T::res)
+    ok = ok && encode_2d(&m_rq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->rq, kb, a.n, kb, 64, BN,
+                         CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (T::h)
+    ok = ok && encode_2d(&m_l1q, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->l1q, kb, a.r, kb, 64, a.h_box,
+                         CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (T::s2)
+    ok = ok && encode_2d(&m_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2t, a.r, a.n,
+                         static_cast<uint64_t>(a.r) * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (T::h_global)
+    ok = ok && encode_2d(&m_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.h_global, a.r, c.b,
+                         static_cast<uint64_t>(a.r) * 2, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+
+  auto kern = twq_gemm_kernel<kMode, BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+  kern<<<grid, kThreads, L::kAlloc, st>>>(m_xq, m_rq, m_l1q, m_l2t, m_h, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmCall& c, cudaStream_t st, int* launches) {
+  if (launches) ++*launches;
+  switch (c.mode) {
+    case kModeFused: return launch_mode<kModeFused, 128>(c, st);
+    case kModeW4A4: return launch_mode<kModeW4A4, 128>(c, st);
+    case kModeLowRank: return launch_mode<kModeLowRank, 128>(c, st);
+    case kModeResF32: return launch_mode<kModeResF32, 128>(c, st);
+    case kModeHOnly: return launch_mode<kModeHOnly, 128>(c, st);
+    case kModeS2F32: return launch_mode<kModeS2F32, 128>(c, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t read_and_clear_device_status(int* code) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  *code = v;
+  return e;
+}
+
+}  // namespace twq

@@ -1,0 +1,45 @@
+// Internal interface between the C-ABI layer (twq_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/twq.h"
+
+namespace twq {
+
+// What one launch of the tensor-core kernel computes.
+enum GemmMode : int {
+  kModeFused = 0,    // Y = bf16(Q(X)Q(R) + bf16(Q(X)Q(L1)) L2)
+  kModeW4A4 = 1,     // Y = bf16(Q(X)Q(R))
+  kModeLowRank = 2,  // Y = bf16(bf16(Q(X)Q(L1)) L2)
+  kModeResF32 = 3,   // out = Q(X)Q(R) in fp32            (unfused comparator, step 1)
+  kModeHOnly = 4,    // out = bf16(Q(X)Q(L1)), b x r      (unfused comparator, step 2)
+  kModeS2F32 = 5,    // out = H L2 in fp32, H read from HBM (unfused comparator, step 3)
+};
+
+struct GemmCall {
+  int mode;
+  const uint8_t* xq;
+  const float* sx;
+  int64_t b;
+  const twq_weights* w;
+  void* out;                // bf16 Y, fp32 b x n, or bf16 H (b x r)
+  const uint16_t* h_global; // kModeS2F32 only: bf16 H, b x r
+};
+
+// Host-side launchers; all return cudaSuccess or the launch error.
+cudaError_t launch_gemm(const GemmCall& call, cudaStream_t stream, int* launches);
+cudaError_t launch_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
+                                float* sx, cudaStream_t stream);
+cudaError_t launch_pack_cols(const uint16_t* w, int64_t m, int64_t cols, uint8_t* q, float* s,
+                             cudaStream_t stream);
+cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out,
+                                  cudaStream_t stream);
+cudaError_t launch_add_cast(const float* a, const float* b, int64_t count, uint16_t* y,
+                            cudaStream_t stream);
+
+// Device status word (first wait site that gave up).
+cudaError_t read_and_clear_device_status(int* code);
+
+}  // namespace twq

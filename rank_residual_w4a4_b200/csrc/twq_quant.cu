@@ -1,0 +1,165 @@
+// Quantization and packing kernels (TwinQuant §2, Eq. (1), groups of 128 along
+// the reduction dimension per §5.1). HBM-bound: 128-bit loads, warp-shuffle
+// absmax, one correctly rounded fp32 division per scale and per element
+// (__fdiv_rn), round half to even (rintf).
+#include <cuda_bf16.h>
+
+#include "twq_internal.h"
+
+namespace twq {
+namespace {
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+
+// Eq. (1) code of v for scale s (s > 0), q_max = 7, as a 4-bit two's-complement nibble.
+__device__ __forceinline__ uint32_t code_nibble(float v, float s) {
+  float t = rintf(__fdiv_rn(v, s));
+  t = fminf(fmaxf(t, -7.0f), 7.0f);
+  return static_cast<uint32_t>(static_cast<int32_t>(t)) & 0xFu;
+}
+
+// One half-warp per (token, group): lane l of the half covers elements
+// [8l, 8l + 8) of the group; a warp covers two consecutive groups of one row.
+__global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x,
+                                                           int64_t b, int m, int64_t ldx,
+                                                           uint8_t* __restrict__ xq,
+                                                           float* __restrict__ sx) {
+  const int G = m / 128;
+  const int pairs = (G + 1) / 2;
+  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = gw / pairs;
+  if (row >= b) return;
+  const int g = static_cast<int>(gw % pairs) * 2 + (lane >> 4);
+  const bool valid = g < G;
+  const int l = lane & 15;
+  uint4 raw = make_uint4(0, 0, 0, 0);
+  if (valid) raw = __ldg(reinterpret_cast<const uint4*>(x + row * ldx + g * 128 + l * 8));
+  float f[8];
+  f[0] = bf16_bits_to_f32(raw.x & 0xFFFFu);
+  f[1] = bf16_bits_to_f32(raw.x >> 16);
+  f[2] = bf16_bits_to_f32(raw.y & 0xFFFFu);
+  f[3] = bf16_bits_to_f32(raw.y >> 16);
+  f[4] = bf16_bits_to_f32(raw.z & 0xFFFFu);
+  f[5] = bf16_bits_to_f32(raw.z >> 16);
+  f[6] = bf16_bits_to_f32(raw.w & 0xFFFFu);
+  f[7] = bf16_bits_to_f32(raw.w >> 16);
+  float a = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(f[k]));
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+  const float s = __fdiv_rn(a, 7.0f);
+  uint32_t word = 0;
+  if (s != 0.0f) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) word |= code_nibble(f[k], s) << (4 * k);
+  }
+  if (valid) {
+    *reinterpret_cast<uint32_t*>(xq + row * (m / 2) + g * 64 + l * 4) = word;
+    if (l == 0) sx[row * G + g] = s;
+  }
+}
+
+// One thread per (group g, column j) of a row-major m x cols BF16 matrix:
+// the group runs down column j (reads are coalesced across j).
+__global__ void __launch_bounds__(128) pack_cols_kernel(const uint16_t* __restrict__ w, int m,
+                                                        int cols, uint8_t* __restrict__ q,
+                                                        float* __restrict__ s) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  const int g = blockIdx.y;
+  if (j >= cols) return;
+  const uint16_t* p = w + static_cast<int64_t>(g) * 128 * cols + j;
+  float a = 0.0f;
+  for (int k = 0; k < 128; ++k) a = fmaxf(a, fabsf(bf16_bits_to_f32(__ldg(p + static_cast<int64_t>(k) * cols))));
+  const float sc = __fdiv_rn(a, 7.0f);
+  s[static_cast<int64_t>(g) * cols + j] = sc;
+  uint4* dst = reinterpret_cast<uint4*>(q + static_cast<int64_t>(j) * (m / 2) + g * 64);
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    uint32_t words[4];
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      uint32_t word = 0;
+      if (sc != 0.0f) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int kk = c * 32 + wi * 8 + k;
+          word |= code_nibble(bf16_bits_to_f32(__ldg(p + static_cast<int64_t>(kk) * cols)), sc)
+                  << (4 * k);
+        }
+      }
+      words[wi] = word;
+    }
+    dst[c] = make_uint4(words[0], words[1], words[2], words[3]);
+  }
+}
+
+// out (cols x rows) = in (rows x cols)^T, 16-bit elements, 32 x 32 tiles.
+__global__ void transpose16_kernel(const uint16_t* __restrict__ in, int rows, int cols,
+                                   uint16_t* __restrict__ out) {
+  __shared__ uint16_t tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = in[static_cast<int64_t>(r) * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) out[static_cast<int64_t>(c) * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+// y = bf16(a + b), elementwise (the unfused comparator's last step).
+__global__ void add_cast_kernel(const float4* __restrict__ a, const float4* __restrict__ b,
+                                int64_t n4, uint2* __restrict__ y) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 u = __ldg(a + i), v = __ldg(b + i);
+    __nv_bfloat162 lo = __floats2bfloat162_rn(u.x + v.x, u.y + v.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(u.z + v.z, u.w + v.w);
+    y[i] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
+                                float* sx, cudaStream_t st) {
+  const int G = static_cast<int>(m / 128);
+  const int64_t warps = b * ((G + 1) / 2);
+  const int64_t blocks = (warps + 7) / 8;
+  quantize_act_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(x, b, static_cast<int>(m),
+                                                                     ldx, xq, sx);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_cols(const uint16_t* w, int64_t m, int64_t cols, uint8_t* q, float* s,
+                             cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>((cols + 127) / 128), static_cast<unsigned>(m / 128));
+  pack_cols_kernel<<<grid, 128, 0, st>>>(w, static_cast<int>(m), static_cast<int>(cols), q, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out,
+                                  cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>((cols + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
+  transpose16_kernel<<<grid, dim3(32, 8), 0, st>>>(in, static_cast<int>(rows),
+                                                    static_cast<int>(cols), out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_add_cast(const float* a, const float* b, int64_t count, uint16_t* y,
+                            cudaStream_t st) {
+  const int64_t n4 = count / 4;
+  int64_t blocks = (n4 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  add_cast_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(a), reinterpret_cast<const float4*>(b), n4,
+      reinterpret_cast<uint2*>(y));
+  return cudaGetLastError();
+}
+
+}  // namespace twq

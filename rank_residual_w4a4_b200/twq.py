@@ -1,0 +1,225 @@
+"""Python binding of libtwq.so (include/twq.h): argument marshalling only.
+
+Each function has the name of the C entry point without the ``twq_`` prefix.
+Tensors are torch CUDA tensors; the binding allocates outputs as the caller
+(the library itself never allocates) and passes the current CUDA stream.
+Every step of the layer runs in the library's kernels; there is no fallback:
+if the library is missing or a tensor is not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtwq.so")
+
+OK = 0
+STATUS_NAMES = {0: "TWQ_OK", 1: "TWQ_ERR_INVALID_ARG", 2: "TWQ_ERR_UNSUPPORTED",
+                3: "TWQ_ERR_MISALIGNED", 4: "TWQ_ERR_CUDA", 5: "TWQ_ERR_NOT_IMPLEMENTED",
+                6: "TWQ_ERR_DEVICE"}
+
+# Every extern "C" symbol that include/twq.h declares.
+EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_sizes",
+           "twq_quantize_act", "twq_pack_weights", "twq_fused_linear", "twq_w4a4_only",
+           "twq_lowrank_only", "twq_unfused_workspace_bytes", "twq_unfused_linear",
+           "twq_device_status", "twq_launches_per_call")
+
+
+class TwqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (what, STATUS_NAMES.get(status, "?"), status))
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [("m", ctypes.c_int64), ("n", ctypes.c_int64), ("r", ctypes.c_int64),
+                ("rq", ctypes.c_void_p), ("sr", ctypes.c_void_p), ("l1q", ctypes.c_void_p),
+                ("sl1", ctypes.c_void_p), ("l2t", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("libtwq.so not found at %s: build it with __graft_entry__.build() "
+                           "or `python rank_residual_w4a4_b200/_build.py`" % path)
+    lib = ctypes.CDLL(path)
+    P, I, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "twq_version": ([], ctypes.c_int),
+        "twq_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "twq_weights_sizes": ([I, I, I, P], ctypes.c_int),
+        "twq_act_sizes": ([I, I, P], ctypes.c_int),
+        "twq_quantize_act": ([P, I, I, I, P, P, P], ctypes.c_int),
+        "twq_pack_weights": ([P, P, P, P, P], ctypes.c_int),
+        "twq_fused_linear": ([P, P, I, P, P, P], ctypes.c_int),
+        "twq_w4a4_only": ([P, P, I, P, P, P], ctypes.c_int),
+        "twq_lowrank_only": ([P, P, I, P, P, P], ctypes.c_int),
+        "twq_unfused_workspace_bytes": ([I, I, I], S),
+        "twq_unfused_linear": ([P, P, I, P, P, P, S, P], ctypes.c_int),
+        "twq_device_status": ([P], ctypes.c_int),
+        "twq_launches_per_call": ([ctypes.c_char_p], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise TwqError(status, what)
+
+
+def _dev(t: torch.Tensor, name: str, dtype) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be on a CUDA device (the library has no CPU path)" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def version() -> int:
+    return load().twq_version()
+
+
+def weights_sizes(m: int, n: int, r: int):
+    arr = (ctypes.c_size_t * 5)()
+    _check(load().twq_weights_sizes(m, n, r, arr), "twq_weights_sizes")
+    return tuple(int(v) for v in arr)
+
+
+def act_sizes(b: int, m: int):
+    arr = (ctypes.c_size_t * 2)()
+    _check(load().twq_act_sizes(b, m, arr), "twq_act_sizes")
+    return tuple(int(v) for v in arr)
+
+
+@dataclass
+class Weights:
+    """Packed weights of one layer (device tensors) in the library's format."""
+    m: int
+    n: int
+    r: int
+    rq: torch.Tensor    # n x m/2 uint8
+    sr: torch.Tensor    # m/128 x n float32
+    l1q: torch.Tensor   # r x m/2 uint8
+    sl1: torch.Tensor   # m/128 x r float32
+    l2t: torch.Tensor   # n x r bfloat16
+
+    def c_struct(self) -> _Weights:
+        nz = lambda t: t.data_ptr() if t.numel() else None
+        return _Weights(self.m, self.n, self.r, self.rq.data_ptr(), self.sr.data_ptr(),
+                        nz(self.l1q), nz(self.sl1), nz(self.l2t))
+
+    @staticmethod
+    def empty(m: int, n: int, r: int, device) -> "Weights":
+        return Weights(m, n, r,
+                       torch.empty((n, m // 2), dtype=torch.uint8, device=device),
+                       torch.empty((m // 128, n), dtype=torch.float32, device=device),
+                       torch.empty((r, m // 2), dtype=torch.uint8, device=device),
+                       torch.empty((m // 128, r), dtype=torch.float32, device=device),
+                       torch.empty((n, r), dtype=torch.bfloat16, device=device))
+
+
+def quantize_act(x: torch.Tensor, xq: torch.Tensor | None = None, sx: torch.Tensor | None = None,
+                 stream=None):
+    """BF16 X (b x m) -> packed codes (b x m/2 uint8) and scales (b x m/128 fp32)."""
+    b, m = x.shape
+    if xq is None:
+        xq = torch.empty((b, m // 2), dtype=torch.uint8, device=x.device)
+    if sx is None:
+        sx = torch.empty((b, max(m // 128, 1)), dtype=torch.float32, device=x.device)
+    _check(load().twq_quantize_act(_dev(x, "x", torch.bfloat16), b, m, m,
+                                   _dev(xq, "xq", torch.uint8), _dev(sx, "sx", torch.float32),
+                                   _stream(stream)), "twq_quantize_act")
+    return xq, sx
+
+
+def pack_weights(R: torch.Tensor, L1: torch.Tensor | None, L2: torch.Tensor | None,
+                 out: Weights | None = None, stream=None) -> Weights:
+    """BF16 R (m x n), L1 (m x r), L2 (r x n) -> packed Weights."""
+    m, n = R.shape
+    r = 0 if L1 is None else L1.shape[1]
+    w = Weights.empty(m, n, r, R.device) if out is None else out
+    cw = w.c_struct()
+    _check(load().twq_pack_weights(
+        _dev(R, "R", torch.bfloat16),
+        _dev(L1, "L1", torch.bfloat16) if r else None,
+        _dev(L2, "L2", torch.bfloat16) if r else None,
+        ctypes.byref(cw), _stream(stream)), "twq_pack_weights")
+    return w
+
+
+def _layer(fn: str, xq, sx, w: Weights, y, stream):
+    b = xq.shape[0]
+    if y is None:
+        y = torch.empty((b, w.n), dtype=torch.bfloat16, device=xq.device)
+    cw = w.c_struct()
+    _check(getattr(load(), fn)(_dev(xq, "xq", torch.uint8), _dev(sx, "sx", torch.float32), b,
+                               ctypes.byref(cw), _dev(y, "y", torch.bfloat16), _stream(stream)), fn)
+    return y
+
+
+def fused_linear(xq, sx, w: Weights, y=None, stream=None):
+    return _layer("twq_fused_linear", xq, sx, w, y, stream)
+
+
+def w4a4_only(xq, sx, w: Weights, y=None, stream=None):
+    return _layer("twq_w4a4_only", xq, sx, w, y, stream)
+
+
+def lowrank_only(xq, sx, w: Weights, y=None, stream=None):
+    return _layer("twq_lowrank_only", xq, sx, w, y, stream)
+
+
+def unfused_workspace_bytes(b: int, n: int, r: int) -> int:
+    return int(load().twq_unfused_workspace_bytes(b, n, r))
+
+
+def unfused_linear(xq, sx, w: Weights, y=None, workspace=None, stream=None):
+    b = xq.shape[0]
+    if y is None:
+        y = torch.empty((b, w.n), dtype=torch.bfloat16, device=xq.device)
+    nbytes = unfused_workspace_bytes(b, w.n, w.r)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=xq.device)
+    cw = w.c_struct()
+    _check(load().twq_unfused_linear(_dev(xq, "xq", torch.uint8), _dev(sx, "sx", torch.float32), b,
+                                     ctypes.byref(cw), _dev(y, "y", torch.bfloat16),
+                                     _dev(workspace, "workspace", torch.uint8),
+                                     workspace.numel(), _stream(stream)), "twq_unfused_linear")
+    return y
+
+
+def device_status() -> int:
+    """Synchronizes; returns 0 or the site code of a kernel wait that ran out."""
+    code = ctypes.c_int(0)
+    st = load().twq_device_status(ctypes.byref(code))
+    if st not in (OK, 6):
+        raise TwqError(st, "twq_device_status")
+    return code.value
+
+
+def launches_per_call(entry_point: str) -> int:
+    return int(load().twq_launches_per_call(entry_point.encode()))

@@ -1,0 +1,217 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Codes and scales must be bit-exact; Y must meet the tolerance in helpers.py.
+Small shapes span several tiles and ragged tails; the five workloads run at
+full size in the launch configuration the benchmark uses, compared on seeded
+row samples where the oracle would be too slow for every row.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from helpers import assert_y_close, bits_of, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def twq(device):
+    from rank_residual_w4a4_b200 import _build, twq as binding
+    _build.build()
+    binding.load()
+    return binding
+
+
+def _status_clean(twq):
+    assert twq.device_status() == 0, "a kernel's bounded wait ran out"
+
+
+def _pack(twq, dev, R, L1, L2):
+    r = 0 if L1 is None else L1.shape[1]
+    return twq.pack_weights(to_dev(R, dev), to_dev(L1, dev) if r else None,
+                            to_dev(L2, dev) if r else None)
+
+
+def _operands(b, m, n, r, seed=0, wl="tiny"):
+    w = synth.WORKLOADS[wl]
+    if m == w.m:
+        x = synth.make_x(w, b=b, seed=seed)
+    else:
+        x = synth.fill(b, m, w.x_dist[0], w.x_dist[1], w.x_dist[2], seed, synth.ID_X)
+    R, L1, L2 = synth.make_weights(w, seed=seed, m=m, n=n, r=r)
+    if r == 0:
+        L1 = L2 = None
+    return x, R, L1, L2
+
+
+# ------------------------------------------------------------- quantize / pack
+
+ADVERSARIAL = {
+    # ties: absmax 7 in lane 0 of each group, x.5 values elsewhere
+    "ties": lambda: np.tile(np.concatenate([[7.0], np.tile(np.arange(-7, 7) + 0.5, 10)[:127]])
+                            .astype(np.float32), (3, 4)),
+    "zero_groups": lambda: np.zeros((5, 512), np.float32),
+    "all_equal": lambda: np.full((4, 256), -0.375, np.float32),
+    "subnormal": lambda: np.tile((np.arange(128) + 1) * np.float32(2.0 ** -133), (2, 2)),
+}
+
+
+def _absmax_lanes():
+    # +-absmax at every lane position (one row per position and sign)
+    rows = []
+    rng = np.random.default_rng(5)
+    for pos in range(128):
+        for sign in (1.0, -1.0):
+            v = rng.uniform(-1, 1, 128).astype(np.float32)
+            v[pos] = sign * 3.0
+            rows.append(v)
+    return np.stack(rows)
+
+
+def _bf16_exact(f):
+    f = np.asarray(f, np.float32)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("case", list(ADVERSARIAL) + ["absmax_lanes"])
+def test_quantize_act_adversarial(twq, device, case):
+    f = _absmax_lanes() if case == "absmax_lanes" else ADVERSARIAL[case]()
+    x = _bf16_exact(f)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    rq, rs = oracle.quantize_act(x)
+    assert np.array_equal(xq.cpu().numpy(), rq)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+
+
+@pytest.mark.parametrize("name,b", [("tiny", 16), ("decode", 1), ("decode", 4), ("decode", 16),
+                                    ("gateup", 2048), ("down", 4096), ("large", 8192),
+                                    ("tiny", 3), ("tiny", 129)])
+def test_quantize_act_bitexact(twq, device, name, b):
+    wl = synth.WORKLOADS[name]
+    x = synth.make_x(wl, b=b)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    rq, rs = oracle.quantize_act(x)
+    assert np.array_equal(xq.cpu().numpy(), rq)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    _status_clean(twq)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "gateup", "down", "large"])
+def test_pack_weights_bitexact(twq, device, name):
+    wl = synth.WORKLOADS[name]
+    R, L1, L2 = synth.make_weights(wl)
+    w = _pack(twq, device, R, L1, L2)
+    ref = oracle.pack_weights(R, L1, L2)
+    assert np.array_equal(w.rq.cpu().numpy(), ref["rq"])
+    assert np.array_equal(w.sr.cpu().numpy().view(np.uint32), ref["sr"].view(np.uint32))
+    assert np.array_equal(w.l1q.cpu().numpy(), ref["l1q"])
+    assert np.array_equal(w.sl1.cpu().numpy().view(np.uint32), ref["sl1"].view(np.uint32))
+    assert np.array_equal(bits_of(w.l2t), ref["l2t"])
+    _status_clean(twq)
+
+
+# ------------------------------------------------------------------ the layer
+
+SHAPES = [  # b, m, n, r: several tiles, ragged b, one/two H chunks, r not a multiple of 64
+    (16, 512, 512, 32), (1, 128, 128, 16), (3, 256, 384, 48), (17, 384, 256, 64),
+    (129, 512, 384, 128), (200, 256, 256, 144), (64, 640, 128, 256), (300, 128, 512, 16),
+]
+
+
+def _oracle_y(x, R, L1, L2, mode, rows=None):
+    return oracle.layer(x, R, L1, L2, mode=mode, rows=rows)["y"]
+
+
+@pytest.mark.parametrize("b,m,n,r", SHAPES)
+def test_fused_matches_oracle(twq, device, b, m, n, r):
+    x, R, L1, L2 = _operands(b, m, n, r, seed=1)
+    w = _pack(twq, device, R, L1, L2)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    y = twq.fused_linear(xq, sx, w)
+    assert_y_close(bits_of(y), _oracle_y(x, R, L1, L2, oracle.FUSED), "fused %s" % ((b, m, n, r),))
+    _status_clean(twq)
+
+
+@pytest.mark.parametrize("b,m,n,r", SHAPES[:5])
+def test_variants_match_oracle(twq, device, b, m, n, r):
+    x, R, L1, L2 = _operands(b, m, n, r, seed=2)
+    w = _pack(twq, device, R, L1, L2)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    y4 = twq.w4a4_only(xq, sx, w)
+    assert_y_close(bits_of(y4), _oracle_y(x, R, L1, L2, oracle.W4A4_ONLY), "w4a4_only")
+    ylr = twq.lowrank_only(xq, sx, w)
+    assert_y_close(bits_of(ylr), _oracle_y(x, R, L1, L2, oracle.LOWRANK_ONLY), "lowrank_only")
+    _status_clean(twq)
+
+
+@pytest.mark.parametrize("b,m,n,r", SHAPES)
+def test_unfused_is_bitwise_fused(twq, device, b, m, n, r):
+    x, R, L1, L2 = _operands(b, m, n, r, seed=3)
+    w = _pack(twq, device, R, L1, L2)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    assert np.array_equal(bits_of(twq.unfused_linear(xq, sx, w)), bits_of(twq.fused_linear(xq, sx, w)))
+    _status_clean(twq)
+
+
+def test_r0_is_w4a4_and_R0_is_lowrank(twq, device):
+    x, R, L1, L2 = _operands(40, 512, 256, 32, seed=4)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    w0 = _pack(twq, device, R, None, None)
+    assert np.array_equal(bits_of(twq.fused_linear(xq, sx, w0)), bits_of(twq.w4a4_only(xq, sx, w0)))
+    wz = _pack(twq, device, np.zeros_like(R), L1, L2)
+    w = _pack(twq, device, R, L1, L2)
+    assert np.array_equal(bits_of(twq.fused_linear(xq, sx, wz)), bits_of(twq.lowrank_only(xq, sx, w)))
+
+
+def test_sign_and_scaling_equivariance(twq, device):
+    x, R, L1, L2 = _operands(24, 512, 256, 0, seed=6)
+    w = _pack(twq, device, R, None, None)
+    y = bits_of(twq.w4a4_only(*twq.quantize_act(to_dev(x, device)), w))
+    yn = bits_of(twq.w4a4_only(*twq.quantize_act(to_dev(x ^ np.uint16(0x8000), device)), w))
+    assert np.array_equal(yn, y ^ np.uint16(0x8000))
+    x2 = _bf16_exact(synth.bf16_to_f32(x) * np.float32(2))
+    y2 = bits_of(twq.w4a4_only(*twq.quantize_act(to_dev(x2, device)), w))
+    assert np.array_equal(synth.bf16_to_f32(y2), synth.bf16_to_f32(y) * np.float32(2))
+
+
+def test_degenerate_inputs(twq, device):
+    b, m, n, r = 33, 256, 128, 16
+    _, R, L1, L2 = _operands(b, m, n, r, seed=7)
+    w = _pack(twq, device, R, L1, L2)
+    xz = np.zeros((b, m), np.uint16)
+    y = bits_of(twq.fused_linear(*twq.quantize_act(to_dev(xz, device)), w))
+    assert not (synth.bf16_to_f32(y) != 0).any()
+    # b == 0 is a no-op that returns an empty result
+    import torch
+    xq0 = torch.empty((0, m // 2), dtype=torch.uint8, device=device)
+    sx0 = torch.empty((0, m // 128), dtype=torch.float32, device=device)
+    assert twq.fused_linear(xq0, sx0, w).shape == (0, n)
+    _status_clean(twq)
+
+
+# --------------------------------------------------- the five workloads, full size
+
+def _full(twq, device, name, b, rows):
+    wl = synth.WORKLOADS[name]
+    x = synth.make_x(wl, b=b)
+    R, L1, L2 = synth.make_weights(wl)
+    w = _pack(twq, device, R, L1, L2)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    y = bits_of(twq.fused_linear(xq, sx, w))
+    rows = np.arange(b) if rows is None else rows
+    ref = _oracle_y(x, R, L1, L2, oracle.FUSED, rows=rows)
+    assert_y_close(y[rows], ref, "%s b=%d" % (name, b))
+    _status_clean(twq)
+    return y, rows
+
+
+@pytest.mark.parametrize("name,b", [("tiny", 16), ("decode", 1), ("decode", 4), ("decode", 16)])
+def test_workload_all_rows(twq, device, name, b):
+    _full(twq, device, name, b, None)
+
+
+@pytest.mark.parametrize("name", ["gateup", "down", "large"])
+def test_workload_sampled_rows(twq, device, name):
+    wl = synth.WORKLOADS[name]
+    _full(twq, device, name, wl.b, synth.sample_rows(wl.b, 24, seed=11))

@@ -155,6 +155,30 @@ TWQ_API twq_status twq_unfused_linear(const uint8_t* xq, const float* sx, int64_
                               twq_stream_t stream);
 
 /*
+ * twq_unfused_linear without a caller-provided workspace, for callers that
+ * may not allocate device memory (for example a plugin whose host framework
+ * owns the whole device-memory budget, or a service that must not let a
+ * cudaMalloc synchronize the device mid-stream). The TwinQuant pages have no
+ * counterpart: this is a convenience of this library.
+ *   Same arguments and result as twq_unfused_linear, minus the workspace.
+ *   Scratch: a fixed 16 MiB array inside the library (a file-scope __device__
+ *   object that every GPU which loads the library holds until the process
+ *   exits). Calls whose twq_unfused_workspace_bytes(b, n, r) exceeds 16 MiB
+ *   return TWQ_ERR_UNSUPPORTED and launch nothing.
+ *   Set-up: the first call on each device resolves the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Sharing: every call uses the same array, which keeps the last call's
+ *   contents. No part of it needs to start at zero (each call writes every
+ *   scratch byte before reading it), but calls that overlap on the GPU (two
+ *   streams, or two host threads) race on it: serialize them.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+TWQ_API twq_status twq_unfused_linear_noalloc(const uint8_t* xq, const float* sx, int64_t b,
+                                              const twq_weights* w, uint16_t* y,
+                                              twq_stream_t stream);
+
+/*
  * Reads and clears the device-side status word (SYNCHRONIZES the device).
  * *code = 0 if no kernel's bounded wait has run out since the last call, else
  * a site code (which wait gave up). Returns TWQ_ERR_DEVICE if *code != 0.

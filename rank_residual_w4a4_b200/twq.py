@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "TWQ_OK", 1: "TWQ_ERR_INVALID_ARG", 2: "TWQ_ERR_UNSUPPORTED",
 EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_sizes",
            "twq_quantize_act", "twq_pack_weights", "twq_fused_linear", "twq_w4a4_only",
            "twq_lowrank_only", "twq_unfused_workspace_bytes", "twq_unfused_linear",
-           "twq_device_status", "twq_launches_per_call")
+           "twq_device_status", "twq_launches_per_call", "twq_unfused_linear_noalloc")
 
 
 class TwqError(RuntimeError):
@@ -68,6 +68,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twq_unfused_linear": ([P, P, I, P, P, P, S, P], ctypes.c_int),
         "twq_device_status": ([P], ctypes.c_int),
         "twq_launches_per_call": ([ctypes.c_char_p], ctypes.c_int),
+        "twq_unfused_linear_noalloc": ([P, P, I, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -210,6 +211,13 @@ def unfused_linear(xq, sx, w: Weights, y=None, workspace=None, stream=None):
                                      _dev(workspace, "workspace", torch.uint8),
                                      workspace.numel(), _stream(stream)), "twq_unfused_linear")
     return y
+
+
+def unfused_linear_noalloc(xq, sx, w: Weights, y=None, stream=None):
+    """twq_unfused_linear with the library's own fixed scratch (no workspace argument);
+    for callers that may not allocate device memory. Calls that overlap on the GPU race
+    on the shared scratch."""
+    return _layer("twq_unfused_linear_noalloc", xq, sx, w, y, stream)
 
 
 def device_status() -> int:

@@ -91,7 +91,7 @@ def load_peaks():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("twq_gemm_sm100.cu", "sm100_ptx.cuh"):
+    for f in ("twq_gemm_sm100.cu", "twq_decode_sm100.cu", "sm100_ptx.cuh"):
         with open(os.path.join(ROOT, "rank_residual_w4a4_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -343,29 +343,23 @@ def run_gpu(args):
     prob.step(0)
     torch.cuda.synchronize()
     gw = capture(prob.step, W)
-    # sampled per-launch events on the launching stream, every 4th step
-    evs = {}
-
-    def timed_step(i):
-        ev = None
-        if i % 4 == 0:
-            ev = (torch.cuda.Event(enable_timing=True, external=True),
-                  torch.cuda.Event(enable_timing=True, external=True))
-            evs[i] = ev
-        prob.step(i, ev=ev)
-
-    gk = capture(timed_step, K)
+    gk = capture(prob.step, K)
     t_load0 = time.time()
-    # keep the GPU busy ~1 s so the clock samples see it under load
-    t_end = time.time() + 1.0
+    # keep the GPU busy for a while so the clock samples see it under load
+    t_end = time.time() + args.clock_seconds
     while time.time() < t_end:
         gw.replay()
         torch.cuda.synchronize()
     elapsed = time_graph(gk, world, device)
     t_load1 = time.time()
     elapsed = max_over_ranks(elapsed, world, device)
-    fused_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in sorted(evs)]
-    t_fused = float(np.mean(fused_ms)) / 1e3
+    # the fused kernel alone: CUDA events around a graph of K back-to-back launches
+    # on the same stream and weight rotation (no events between launches, which
+    # would serialize them)
+    def fused_only(i):
+        c = i % prob.copies
+        twq.fused_linear(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c])
+    t_fused = kernel_only_time(prob, fused_only, K)
     st = twq.device_status()
     if st != 0:
         raise RuntimeError("device wait timed out at site %d" % st)
@@ -396,9 +390,11 @@ def run_gpu(args):
                    "step": "twq_quantize_act + twq_fused_linear",
                    "l2": "weights rotate over %d copies (%.0f MB > 2x L2)" % (
                        prob.copies, prob.copies * weight_bytes(wl.m, wl.n, wl.r) / 1e6),
-                   "launch": "CUDA graph of the K timed steps"},
+                   "launch": "CUDA graph of the K timed steps; the fused kernel is "
+                             "launched with programmatic stream serialization"},
         "effective_tops": round(ops * world * K / elapsed / 1e12, 3),
         "fused_kernel_us": round(t_fused * 1e6, 3),
+        "fused_kernel_timing": "events around a graph of K back-to-back fused launches",
         "roofline": roofline_entry(name, t_fused, peaks, profiled_traffic(name)),
         "e2e": e2e,
         "gpu_launches": 2 * K,
@@ -605,6 +601,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--clock-seconds", type=float, default=1.0,
+                    help="seconds of warm-up replays before the timed region (clock sampling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -130,6 +130,13 @@ TWQ_API twq_status twq_pack_weights(const uint16_t* R, const uint16_t* L1, const
  * stage 2 against L2, and writes Y once.
  *   xq, sx  from twq_quantize_act;  w  from twq_pack_weights;  y  b x n BF16 (output)
  * w->r == 0 gives exactly the twq_w4a4_only result.
+ * Decode shapes (b <= 16) run a split-K kernel launched with programmatic
+ * stream serialization: when the kernel just before it on the stream signals
+ * programmatic completion early (twq_quantize_act does), its prologue and its
+ * reads of the packed weights start while that kernel is still running, and
+ * its reads of xq / sx wait until that kernel has completed. So xq / sx may come
+ * from the preceding kernel, but the weights must not be written by a kernel
+ * that signals early (twq_pack_weights does not).
  */
 TWQ_API twq_status twq_fused_linear(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
                             uint16_t* y, twq_stream_t stream);

@@ -15,7 +15,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libtwq.so")
-SOURCES = ["twq_api.cu", "twq_gemm_sm100.cu", "twq_quant.cu", "twq_noalloc.cu"]
+SOURCES = ["twq_api.cu", "twq_gemm_sm100.cu", "twq_decode_sm100.cu", "twq_quant.cu",
+           "twq_noalloc.cu"]
 HEADERS = ["sm100_ptx.cuh", "twq_internal.h"]
 
 NVCC_FLAGS = [

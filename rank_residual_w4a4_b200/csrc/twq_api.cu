@@ -49,7 +49,9 @@ twq_status check_layer(const uint8_t* xq, const float* sx, int64_t b, const twq_
 twq_status run(int mode, const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
                void* out, const uint16_t* h, twq_stream_t stream) {
   twq::GemmCall c{mode, xq, sx, b, w, out, h};
-  return from_cuda(twq::launch_gemm(c, reinterpret_cast<cudaStream_t>(stream), nullptr));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (twq::decode_eligible(c)) return from_cuda(twq::launch_decode(c, st));
+  return from_cuda(twq::launch_gemm(c, st, nullptr));
 }
 
 }  // namespace
@@ -178,8 +180,11 @@ twq_status twq_device_status(int* code) {
   if (!code) return TWQ_ERR_INVALID_ARG;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return TWQ_ERR_CUDA;
-  e = twq::read_and_clear_device_status(code);
+  int c1 = 0, c2 = 0;
+  e = twq::read_and_clear_device_status(&c1);
+  if (e == cudaSuccess) e = twq::read_and_clear_decode_status(&c2);
   if (e != cudaSuccess) return TWQ_ERR_CUDA;
+  *code = c1 ? c1 : c2;
   return *code ? TWQ_ERR_DEVICE : TWQ_OK;
 }
 

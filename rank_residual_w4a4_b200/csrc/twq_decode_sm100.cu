@@ -1,0 +1,672 @@
+// Decode-shape kernel (b <= 16 tokens) of the dual-component W4A4 + low-rank
+// layer for sm_100a (TwinQuant, "Learnable Subspace Decomposition for 4-Bit
+// LLM Quantization", §4.3 and Fig. 4; same arithmetic as twq_gemm_sm100.cu).
+//
+// With a handful of tokens the layer is a stream of the packed weights, so the
+// kernel is laid out for HBM rather than for the tensor cores:
+//   * swap-AB: the 128 output columns of a tile are the MMA's M side, the
+//     tokens (padded to 16) its N side;
+//   * split K: a cluster of KS CTAs shares one column tile; CTA k of the cluster
+//     reduces over its own m/KS slice of the groups, so 4 x (n/128) CTAs stream
+//     the weights at once;
+//   * R codes: every group tile of the CTA is requested by TMA at once (64-byte
+//     swizzle); warps unpack them in registers and write the int8 A operand
+//     straight into tensor memory (tcgen05.st), so shared memory only carries
+//     the packed bytes once;
+//   * L1 codes (mostly L2-resident after the first cluster) are loaded with
+//     plain loads into tensor memory the same way;
+//   * stage 1 gives each CTA a partial H (its groups) for all r; the partials
+//     are pushed over distributed shared memory to the CTA that owns each
+//     16-column unit of r, which sums them in a fixed order, rounds to BF16 and
+//     runs its unit's share of stage 2 (H kept on chip, never in HBM);
+//   * Y partials (residual over the CTA's groups + stage 2 over its r units)
+//     are pushed to the CTA that owns each column slice, summed in a fixed
+//     order, rounded to BF16 and stored once.
+// Cross-CTA data moves only as st.async pushes into the receiving CTA's shared
+// memory, each completing bytes on the receiver's mbarrier (which registered
+// the exact byte count it expects before the cluster rendezvous). A CTA never
+// reads a peer's shared memory, and every write into it has landed once its
+// bounded wait completes, so no CTA exits while a peer may still write into it.
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+#include "twq_internal.h"
+
+namespace twq {
+
+__device__ int g_decode_status;
+
+
+namespace {
+
+constexpr int kThreads = 640;        // 20 warps
+constexpr int kNT = 16;               // token tile: N of every MMA
+constexpr int kMaxGroups = 8;         // groups of 128 per CTA
+constexpr int kRing = 4;              // tensor-memory ring depth (operands and accumulators)
+constexpr int kTmemCols = 512;
+constexpr int kColL1 = 0;             // kRing x 32: int8 L1 operand tiles
+constexpr int kColR = 128;            // kRing x 32: int8 R operand tiles
+constexpr int kColDh = 256;           // kMaxGroups x 16: stage-1 accumulators
+constexpr int kColDres = 384;         // kMaxGroups x 16: residual accumulators
+constexpr int kColDlr = 0;            // 16: stage-2 accumulator (L1 ring, free after stage 1)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+enum DecodeSite : int {
+  kDSiteX = 21, kDSiteR = 22, kDSiteL1 = 23, kDSiteAl = 24, kDSiteH = 25, kDSiteRes = 26,
+  kDSiteAr = 27, kDSiteHReady = 28, kDSiteHb = 29, kDSiteL2 = 30, kDSiteLr = 31,
+  kDSiteYReady = 32, kDSiteFinal = 33,
+};
+
+template <int kMode>
+struct DTraits {
+  static constexpr bool res = kMode == kModeFused || kMode == kModeW4A4;
+  static constexpr bool lr = kMode == kModeFused || kMode == kModeLowRank;
+};
+
+struct DecodeArgs {
+  const float* sx;
+  const float* sr;
+  const float* sl1;
+  uint16_t* y;
+  int64_t b;
+  int m, n, r, G;
+};
+
+struct DLayout {
+  static constexpr int kOffR = 0;                              // kMaxGroups x 8 KB (SW64)
+  static constexpr int kOffL1 = kOffR + kMaxGroups * 8192;     // kMaxGroups x 8 KB (SW64)
+  static constexpr int kOffXu = kOffL1 + kMaxGroups * 8192;    // kMaxGroups x 2 KB (SW128)
+  static constexpr int kOffL2 = kOffXu + kMaxGroups * 2048;    // 16 KB (SW128)
+  static constexpr int kOffHb = kOffL2 + 16384;                // 2 KB (SW128)
+  static constexpr int kOffXp = kOffHb + 2048;                 // kMaxGroups x 1 KB
+  static constexpr int kOffSx = kOffXp + kMaxGroups * 1024;    // [group][token] fp32
+  static constexpr int kOffHred = kOffSx + kMaxGroups * kNT * 4;
+  static constexpr int kHredBytes = 128 * kNT * 4;             // [src][c][t], KS * slice <= 128
+  static constexpr int kOffYred = kOffHred + kHredBytes;
+  static constexpr int kYredBytes = 128 * kNT * 4;             // [src][j][t], KS * cols = 128
+  static constexpr int kOffBar = kOffYred + kYredBytes;
+  static constexpr int kNumBars = 64;
+  static constexpr int kBytes = kOffBar + kNumBars * 8 + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+static_assert(DLayout::kAlloc <= 227 * 1024, "shared memory budget");
+
+__device__ __forceinline__ void d_fail(int site) { atomicCAS(&g_decode_status, 0, site); }
+
+template <bool kCluster>
+__device__ __noinline__ bool d_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                    int site) {
+  auto probe = [&]() {
+    return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (probe()) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (probe()) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      d_fail(site);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint8_t* d_align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ uint32_t d_sw128(int row, int c) {
+  return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
+}
+
+// 8 packed bytes (16 codes) -> 16 int8 bytes holding 16*q; even-index codes first.
+__device__ __forceinline__ void unpack8(uint32_t lo, uint32_t hi, uint32_t* o) {
+  o[0] = (lo << 4) & 0xF0F0F0F0u;
+  o[1] = lo & 0xF0F0F0F0u;
+  o[2] = (hi << 4) & 0xF0F0F0F0u;
+  o[3] = hi & 0xF0F0F0F0u;
+}
+
+// Row j of a TMA tile of 64-byte rows in the 64-byte swizzle -> 32 words of int8
+// codes (16*q), stored into tensor-memory lane j, 32 columns from `col`.
+__device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int j, uint32_t taddr) {
+  const uint8_t* row = tile + j * 64;
+  const int sw = (j >> 1) & 3;
+  uint32_t v[32];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
+    unpack8(w.x, w.y, &v[c * 8]);
+    unpack8(w.z, w.w, &v[c * 8 + 4]);
+  }
+  tmem_st32(taddr, v);
+}
+
+// Range of 16-column units of r owned by cluster rank k.
+__device__ __forceinline__ void unit_range(int U, int KS, int k, int& u0, int& u1) {
+  u0 = k * U / KS;
+  u1 = (k + 1) * U / KS;
+}
+
+template <int kMode, int KS>
+__global__ void __launch_bounds__(kThreads, 1)
+    twq_decode_kernel(const __grid_constant__ CUtensorMap tm_rq,
+                      const __grid_constant__ CUtensorMap tm_l1q,
+                      const __grid_constant__ CUtensorMap tm_xq,
+                      const __grid_constant__ CUtensorMap tm_l2t, const DecodeArgs args) {
+  using L = DLayout;
+  using T = DTraits<kMode>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_abort;
+  uint8_t* smem = d_align1024(smem_raw);
+  uint8_t* rtiles = smem + L::kOffR;
+  uint8_t* ltiles = smem + L::kOffL1;
+  uint8_t* xu = smem + L::kOffXu;
+  uint8_t* l2s = smem + L::kOffL2;
+  uint8_t* hbs = smem + L::kOffHb;
+  uint8_t* xp = smem + L::kOffXp;
+  float* sxs = reinterpret_cast<float*>(smem + L::kOffSx);
+  float* hred = reinterpret_cast<float*>(smem + L::kOffHred);
+  float* yred = reinterpret_cast<float*>(smem + L::kOffYred);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* rfull = bars;                     // [kMaxGroups] TMA of R tiles
+  uint64_t* lfull = rfull + kMaxGroups;       // [kMaxGroups] TMA of L1 tiles
+  uint64_t* al_full = lfull + kMaxGroups;     // [kRing] L1 operand slot written
+  uint64_t* al_empty = al_full + kRing;       // [kRing] L1 operand slot read by the MMA
+  uint64_t* ar_full = al_empty + kRing;       // [kRing] R operand slot written
+  uint64_t* ar_empty = ar_full + kRing;       // [kRing]
+  uint64_t* h_full = ar_empty + kRing;        // [kMaxGroups] stage-1 accumulator ready
+  uint64_t* res_full = h_full + kMaxGroups;   // [kMaxGroups] residual accumulator ready
+  uint64_t* xfull = res_full + kMaxGroups;
+  uint64_t* xready = xfull + 1;
+  uint64_t* l2full = xready + 1;
+  uint64_t* hb_ready = l2full + 1;
+  uint64_t* lr_full = hb_ready + 1;
+  uint64_t* h_ready = lr_full + 1;
+  uint64_t* y_ready = h_ready + 1;
+  uint64_t* mma_done = y_ready + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
+  volatile int* abort_flag = &s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ks = static_cast<int>(cluster_rank());
+  const int n0 = blockIdx.y * 128;
+  const int G = args.G;
+  const int g0 = ks * G / KS;
+  const int ng = (ks + 1) * G / KS - g0;
+  const int U = args.r / 16;
+  int u0 = 0, u1 = 0;
+  if (T::lr) unit_range(U, KS, ks, u0, u1);
+  const int my_units = u1 - u0;
+  constexpr int kColsPerOwner = 128 / KS;
+  constexpr int kHSlice = 128 / KS;  // r <= 128 here: at most 128/KS columns of r per CTA
+
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&tm_rq);
+    tma_prefetch_desc(&tm_l1q);
+    tma_prefetch_desc(&tm_xq);
+    tma_prefetch_desc(&tm_l2t);
+  }
+  if (warp == 0) {
+    // barrier init spread over the warp: lane i owns group i's copy barriers
+    if (lane < kMaxGroups) {
+      mbar_init(&rfull[lane], 1);
+      mbar_init(&lfull[lane], 1);
+      mbar_init(&h_full[lane], 1);
+      mbar_init(&res_full[lane], 1);
+    }
+    if (lane < kRing) {
+      mbar_init(&al_full[lane], 4);
+      mbar_init(&al_empty[lane], 1);
+      mbar_init(&ar_full[lane], 4);
+      mbar_init(&ar_empty[lane], 1);
+    }
+    if (lane == 31) {
+      mbar_init(xfull, 1);
+      mbar_init(xready, 2);
+      mbar_init(l2full, 1);
+      mbar_init(hb_ready, 4);
+      mbar_init(lr_full, 1);
+      // Exchange barriers complete on bytes: this CTA expects every peer's partials
+      // for the r units and the column slice it owns (registered before the
+      // cluster rendezvous, so before any peer can send).
+      mbar_init(h_ready, 1);
+      mbar_init(y_ready, 1);
+      mbar_arrive_expect_tx(h_ready, KS * my_units * 16 * kNT * 4);
+      mbar_arrive_expect_tx(y_ready, KS * kColsPerOwner * kNT * 4);
+      mbar_init(mma_done, 1);
+      mbar_init(mma_done + 1, 1);
+      s_abort = 0;
+    }
+    fence_barrier_init();
+    __syncwarp();
+    // Every copy of this CTA is requested before the cluster rendezvous (TMA writes
+    // only this CTA's shared memory and completes on its own barriers): lane gi
+    // issues group gi's tiles.
+    if (lane < ng) {
+      const int gi = lane;
+      if (T::lr) {
+        mbar_arrive_expect_tx(&lfull[gi], 8192);
+        tma_load_2d(ltiles + gi * 8192, &tm_l1q, &lfull[gi], (g0 + gi) * 64, 0);
+      }
+      if (T::res) {
+        mbar_arrive_expect_tx(&rfull[gi], 8192);
+        tma_load_2d(rtiles + gi * 8192, &tm_rq, &rfull[gi], (g0 + gi) * 64, n0);
+      }
+    }
+    if (lane == 31) {
+      if (T::lr && my_units > 0) {
+        mbar_arrive_expect_tx(l2full, 16384);
+        tma_load_2d(l2s, &tm_l2t, l2full, u0 * 16, n0);
+      }
+      // The activation codes may come from the kernel just before this one on the
+      // stream (launched with programmatic serialization): wait for it first.
+      pdl_wait();
+      mbar_arrive_expect_tx(xfull, ng * 1024);
+      for (int gi = 0; gi < ng; ++gi) tma_load_2d(xp + gi * 1024, &tm_xq, xfull, (g0 + gi) * 64, 0);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  // Every CTA of the cluster has initialized its barriers before any peer
+  // writes into its shared memory or arrives on its barriers.
+  cluster_sync_startup();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------ residual MMA issuer (lane 0 of warp 0)
+    if (lane == 0) {
+      bool ok = d_wait<false>(xready, 0, abort_flag, kDSiteX);
+      const uint32_t xu0 = smem_u32(xu);
+      const uint32_t idesc = idesc_i8(kNT);
+      if (T::res) {
+        for (int gi = 0; gi < ng && ok; ++gi) {
+          const int slot = gi % kRing;
+          const uint32_t ph = (gi / kRing) & 1;
+          const uint64_t db = smem_desc_sw128(xu0 + gi * 2048);
+          if (!(ok = d_wait<false>(&ar_full[slot], ph, abort_flag, kDSiteAr))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_i8_tmem_a(tmem_base + kColDres + gi * 16, tmem_base + kColR + slot * 32 + k * 8,
+                          db + 2 * k, idesc, k > 0);
+          mma_commit(&ar_empty[slot]);
+          mma_commit(&res_full[gi]);
+        }
+      }
+      mma_commit(mma_done + 1);
+      // The CTA waits for its own copies and MMAs before it can finish.
+      int never = 0;
+      d_wait<false>(mma_done + 1, 0, &never, kDSiteFinal);
+      d_wait<false>(xfull, 0, &never, kDSiteFinal);
+      for (int gi = 0; gi < ng; ++gi) {
+        if (T::lr) d_wait<false>(&lfull[gi], 0, &never, kDSiteFinal);
+        if (T::res) d_wait<false>(&rfull[gi], 0, &never, kDSiteFinal);
+      }
+      if (T::lr && my_units > 0) d_wait<false>(l2full, 0, &never, kDSiteFinal);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = d_wait<false>(xready, 0, abort_flag, kDSiteX);
+      const uint32_t xu0 = smem_u32(xu);
+      const uint32_t idesc = idesc_i8(kNT);
+      for (int gi = 0; gi < ng && ok; ++gi) {
+        const int slot = gi % kRing;
+        const uint32_t ph = (gi / kRing) & 1;
+        const uint64_t db = smem_desc_sw128(xu0 + gi * 2048);
+        if (T::lr) {
+          if (!(ok = d_wait<false>(&al_full[slot], ph, abort_flag, kDSiteAl))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_i8_tmem_a(tmem_base + kColDh + gi * 16, tmem_base + kColL1 + slot * 32 + k * 8,
+                          db + 2 * k, idesc, k > 0);
+          mma_commit(&al_empty[slot]);
+          mma_commit(&h_full[gi]);
+        }
+      }
+      if (T::lr && my_units > 0 && ok) {
+        ok = d_wait<true>(hb_ready, 0, abort_flag, kDSiteHb) &&
+             d_wait<false>(l2full, 0, abort_flag, kDSiteL2);
+        if (ok) {
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(smem_u32(l2s));
+          const uint64_t db = smem_desc_sw128(smem_u32(hbs));
+          for (int u = 0; u < my_units; ++u)
+            mma_bf16(tmem_base + kColDlr, da + 2 * u, db + 2 * u, idesc_bf16(kNT), u > 0);
+          mma_commit(lr_full);
+        }
+      }
+      mma_commit(mma_done);
+      int never = 0;
+      d_wait<false>(mma_done, 0, &never, kDSiteFinal);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------ X unpack (warps 2 and 3)
+    const int tid = threadIdx.x - 64;
+    pdl_wait();    // the scales, like the codes, may come from the preceding kernel
+    float sxv[2];  // activation scales, loaded before the codes arrive
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int e = tid + 64 * i;
+      const int gi = e / kNT, t = e % kNT;
+      sxv[i] = (gi < ng && t < args.b) ? __ldg(args.sx + static_cast<int64_t>(t) * G + g0 + gi) : 0.0f;
+    }
+    if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) {
+      for (int e = tid; e < ng * kNT * 8; e += 64) {
+        const int gi = e / (kNT * 8);
+        const int row = (e / 8) % kNT;
+        const int c = e & 7;
+        const uint2 w = *reinterpret_cast<const uint2*>(xp + gi * 1024 + row * 64 + c * 8);
+        uint32_t o[4];
+        unpack8(w.x, w.y, o);
+        *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(row, c)) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) sxs[tid + 64 * i] = sxv[i];
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xready);
+    }
+  } else if (warp < 12) {
+    // -------- operand tiles -> tensor memory: L1 (warps 4-7) and R (warps 8-11)
+    const bool is_l1 = warp < 8;
+    const int q = warp & 3;
+    const int j = q * 32 + lane;  // tensor-memory lane: r index for L1, column for R
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    if (is_l1 ? T::lr : T::res) {
+      uint64_t* tfull = is_l1 ? lfull : rfull;
+      uint64_t* sfull = is_l1 ? al_full : ar_full;
+      uint64_t* sempty = is_l1 ? al_empty : ar_empty;
+      const uint8_t* tiles = is_l1 ? ltiles : rtiles;
+      const int col0 = is_l1 ? kColL1 : kColR;
+      for (int gi = 0; gi < ng; ++gi) {
+        const int slot = gi % kRing;
+        const uint32_t ph = (gi / kRing) & 1;
+        if (!d_wait<false>(&tfull[gi], 0, abort_flag, is_l1 ? kDSiteL1 : kDSiteR)) break;
+        if (!d_wait<false>(&sempty[slot], ph ^ 1u, abort_flag, is_l1 ? kDSiteAl : kDSiteAr)) break;
+        tc_fence_after();
+        tile_row_to_tmem(tiles + gi * 8192, j, tmem_base + lane_addr + col0 + slot * 32);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfull[slot]);
+      }
+    }
+  } else if (warp < 16) {
+    // --------------- stage-1 drain, H exchange, BF16 H for stage 2 (warps 12-15)
+    if (T::lr) {
+      const int q = warp & 3;
+      const int c = q * 32 + lane;  // index into r
+      const bool c_ok = c < args.r;
+      const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+      float sl1v[kMaxGroups];
+#pragma unroll
+      for (int gi = 0; gi < kMaxGroups; ++gi)
+        sl1v[gi] = (gi < ng && c_ok) ? __ldg(args.sl1 + static_cast<int64_t>(g0 + gi) * args.r + c) : 0.0f;
+      float acc[kNT];
+#pragma unroll
+      for (int t = 0; t < kNT; ++t) acc[t] = 0.0f;
+      bool ok = d_wait<false>(xready, 0, abort_flag, kDSiteX);
+#pragma unroll
+      for (int gi = 0; gi < kMaxGroups; ++gi) {
+        if (gi < ng && ok) {
+          if (!(ok = d_wait<false>(&h_full[gi], 0, abort_flag, kDSiteH))) break;
+          tc_fence_after();
+          uint32_t v[16];
+          tmem_ld16(tmem_base + lane_addr + kColDh + gi * 16, v);
+          tmem_wait_ld();
+          const float* sxg = sxs + gi * kNT;
+#pragma unroll
+          for (int t = 0; t < kNT; ++t)
+            acc[t] = fmaf(static_cast<float>(static_cast<int32_t>(v[t])) * sl1v[gi], sxg[t], acc[t]);
+        }
+      }
+      tc_fence_before();
+      // push this CTA's partial H for row c to the owner of c's 16-column unit
+      // (pushed even after a local failure, so the exchange stays complete)
+      if (c_ok) {
+        const int u = c / 16;
+        int owner = 0, ou0 = 0;
+        for (int k = 0; k < KS; ++k) {
+          int a0, a1;
+          unit_range(U, KS, k, a0, a1);
+          if (u >= a0 && u < a1) {
+            owner = k;
+            ou0 = a0;
+          }
+        }
+        const int cl = c - ou0 * 16;
+        const uint32_t dst = map_peer(smem_u32(hred + (ks * kHSlice + cl) * kNT), owner);
+        const uint32_t rbar = map_peer(smem_u32(h_ready), owner);
+#pragma unroll
+        for (int t = 0; t < kNT; t += 4)
+          st_async_peer_v4(dst + t * 4, acc[t] * 0.00390625f, acc[t + 1] * 0.00390625f,
+                           acc[t + 2] * 0.00390625f, acc[t + 3] * 0.00390625f, rbar);
+      }
+      // An owner waits until every peer's bytes have landed (so none is still writing
+      // into it when it exits); the wait ignores the abort flag for the same reason.
+      int keep_waiting = 0;
+      const bool got = my_units > 0 ? d_wait<true>(h_ready, 0, &keep_waiting, kDSiteHReady) : true;
+      if (ok && got && my_units > 0) {
+        const int tid = threadIdx.x - 384;
+        const int slice = my_units * 16;
+        for (int e = tid; e < slice * kNT; e += 128) {
+          const int cl = e / kNT, t = e % kNT;
+          float h = 0.0f;
+          for (int k = 0; k < KS; ++k) h += hred[(k * kHSlice + cl) * kNT + t];
+          *reinterpret_cast<__nv_bfloat16*>(hbs + d_sw128(t, cl >> 3) + (cl & 7) * 2) =
+              __float2bfloat16_rn(h);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hb_ready);
+      }
+    }
+  } else {
+    // ------------------------------- residual drain, Y exchange, store (warps 16-19)
+    const int q = warp & 3;
+    const int j = q * 32 + lane;  // column of the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    float acc[kNT];
+#pragma unroll
+    for (int t = 0; t < kNT; ++t) acc[t] = 0.0f;
+    bool ok = d_wait<false>(xready, 0, abort_flag, kDSiteX);
+    if (T::res) {
+      float srv[kMaxGroups];
+#pragma unroll
+      for (int gi = 0; gi < kMaxGroups; ++gi)
+        srv[gi] = gi < ng ? __ldg(args.sr + static_cast<int64_t>(g0 + gi) * args.n + n0 + j) : 0.0f;
+#pragma unroll
+      for (int gi = 0; gi < kMaxGroups; ++gi) {
+        if (gi < ng && ok) {
+          if (!(ok = d_wait<false>(&res_full[gi], 0, abort_flag, kDSiteRes))) break;
+          tc_fence_after();
+          uint32_t v[16];
+          tmem_ld16(tmem_base + lane_addr + kColDres + gi * 16, v);
+          tmem_wait_ld();
+          const float* sxg = sxs + gi * kNT;
+#pragma unroll
+          for (int t = 0; t < kNT; ++t)
+            acc[t] = fmaf(static_cast<float>(static_cast<int32_t>(v[t])) * srv[gi], sxg[t], acc[t]);
+        }
+      }
+    }
+    float part[kNT];
+#pragma unroll
+    for (int t = 0; t < kNT; ++t) part[t] = acc[t] * 0.00390625f;
+    if (T::lr && my_units > 0 && ok) {
+      if ((ok = d_wait<false>(lr_full, 0, abort_flag, kDSiteLr))) {
+        tc_fence_after();
+        uint32_t v[16];
+        tmem_ld16(tmem_base + lane_addr + kColDlr, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < kNT; ++t) part[t] += __uint_as_float(v[t]);
+      }
+    }
+    tc_fence_before();
+    {  // push the partial of column j to the CTA that finalizes j's slice (always)
+      const int owner = j / kColsPerOwner;
+      const int jl = j % kColsPerOwner;
+      const uint32_t dst = map_peer(smem_u32(yred + (ks * kColsPerOwner + jl) * kNT), owner);
+      const uint32_t rbar = map_peer(smem_u32(y_ready), owner);
+#pragma unroll
+      for (int t = 0; t < kNT; t += 4)
+        st_async_peer_v4(dst + t * 4, part[t], part[t + 1], part[t + 2], part[t + 3], rbar);
+    }
+    int keep_waiting = 0;  // not the abort flag: peers may still be writing into this CTA
+    const bool got = d_wait<true>(y_ready, 0, &keep_waiting, kDSiteYReady);
+    if (ok && got) {
+      const int tid = threadIdx.x - 512;
+      for (int e = tid; e < kColsPerOwner * kNT; e += 128) {
+        const int t = e / kColsPerOwner, jl = e % kColsPerOwner;
+        float yv = 0.0f;
+        for (int k = 0; k < KS; ++k) yv += yred[(k * kColsPerOwner + jl) * kNT + t];
+        if (t < args.b)
+          args.y[static_cast<int64_t>(t) * args.n + n0 + ks * kColsPerOwner + jl] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(yv));
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn d_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool d_encode(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+              uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = d_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int kMode, int KS>
+cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
+  const twq_weights* w = c.w;
+  DecodeArgs a{};
+  a.sx = c.sx;
+  a.sr = w->sr;
+  a.sl1 = w->sl1;
+  a.y = static_cast<uint16_t*>(c.out);
+  a.b = c.b;
+  a.m = static_cast<int>(w->m);
+  a.n = static_cast<int>(w->n);
+  a.r = static_cast<int>(w->r);
+  a.G = a.m / 128;
+  CUtensorMap m_rq{}, m_l1q{}, m_xq{}, m_l2t{};
+  const uint64_t kb = static_cast<uint64_t>(a.m / 2);
+  bool ok = d_encode(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, kb, c.b, kb, 64, kNT,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (DTraits<kMode>::res)
+    ok = ok && d_encode(&m_rq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->rq, kb, a.n, kb, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
+  if (DTraits<kMode>::lr)
+    ok = ok && d_encode(&m_l1q, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->l1q, kb, a.r, kb, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
+  if (DTraits<kMode>::lr)
+    ok = ok && d_encode(&m_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2t, a.r, a.n,
+                        static_cast<uint64_t>(a.r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  auto kern = twq_decode_kernel<kMode, KS>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DLayout::kAlloc);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(KS, a.n / 128, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = DLayout::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = KS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  // Programmatic stream serialization: if the preceding kernel signals early
+  // (twq_quantize_act does), this kernel's prologue and weight loads overlap it;
+  // the activation reads wait for its completion (griddepcontrol.wait).
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, kern, m_rq, m_l1q, m_xq, m_l2t, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_eligible(const GemmCall& c) {
+  const twq_weights* w = c.w;
+  if (c.mode != kModeFused && c.mode != kModeW4A4 && c.mode != kModeLowRank) return false;
+  if (c.b < 1 || c.b > kNT) return false;
+  if (c.mode != kModeW4A4 && (w->r <= 0 || w->r > 128)) return false;
+  const int64_t G = w->m / 128;
+  return G <= 8 * kMaxGroups && w->n % 128 == 0;
+}
+
+cudaError_t launch_decode(const GemmCall& c, cudaStream_t st) {
+  const int64_t G = c.w->m / 128;
+  const bool ks8 = G > 4 * kMaxGroups;
+  switch (c.mode) {
+    case kModeFused:
+      return ks8 ? launch_decode_mode<kModeFused, 8>(c, st) : launch_decode_mode<kModeFused, 4>(c, st);
+    case kModeW4A4:
+      return ks8 ? launch_decode_mode<kModeW4A4, 8>(c, st) : launch_decode_mode<kModeW4A4, 4>(c, st);
+    case kModeLowRank:
+      return ks8 ? launch_decode_mode<kModeLowRank, 8>(c, st)
+                 : launch_decode_mode<kModeLowRank, 4>(c, st);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t read_and_clear_decode_status(int* code) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_decode_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_decode_status, &zero, sizeof(int));
+  *code = v;
+  return e;
+}
+
+}  // namespace twq

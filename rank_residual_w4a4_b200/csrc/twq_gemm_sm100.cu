@@ -37,10 +37,12 @@ __device__ int g_device_status;
 namespace {
 
 constexpr int kThreads = 512;
+
 constexpr int kBM = 128;
 constexpr int kPackedStages = 4;
 constexpr int kUnpackedStages = 2;
-constexpr int kScaleSlots = 4;
+constexpr int kScaleSlots = 8;
+constexpr int kAccBufs = 4;     // TMEM accumulator buffers (BN columns each)
 constexpr int kHChunk = 128;  // H columns per stage-1 pass
 constexpr int kMaxRank = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a wait that lasts 2 s is a failure
@@ -69,10 +71,11 @@ struct SmemLayout {
   static constexpr int kOffHb = kOffU + kUnpackedStages * kUStage;
   static constexpr int kOffScale = kOffHb + kHb;
   static constexpr int kOffBar = kOffScale + kScaleSlots * kScaleSlot;
-  static constexpr int kNumBars = 2 * kPackedStages + 2 * kUnpackedStages + 4 + 2 * kScaleSlots + 3;
+  static constexpr int kNumBars =
+      2 * kPackedStages + 2 * kUnpackedStages + 2 * kAccBufs + 2 * kScaleSlots + 3;
   static constexpr int kBytes = kOffBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
-  static constexpr int kTmemCols = 2 * BN;      // two accumulator buffers
+  static constexpr int kTmemCols = kAccBufs * BN;  // accumulator buffers
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
   static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of 2");
 };
@@ -227,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* ufull = empty + kPackedStages;
   uint64_t* uempty = ufull + kUnpackedStages;
   uint64_t* acc_full = uempty + kUnpackedStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* sc_full = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + kAccBufs;
+  uint64_t* sc_full = acc_empty + kAccBufs;
   uint64_t* sc_empty = sc_full + kScaleSlots;
   uint64_t* hb_ready = sc_empty + kScaleSlots;
   uint64_t* hb_free = hb_ready + 1;
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ufull[i], 4);
       mbar_init(&uempty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 8);
     }
@@ -415,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_commit(&uempty[u.idx]);
               mma_commit(&acc_full[a.idx]);
               u.next(kUnpackedStages);
-              a.next(2);
+              a.next(kAccBufs);
             }
           }
         }
@@ -434,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&uempty[u.idx]);
             mma_commit(&acc_full[a.idx]);
             u.next(kUnpackedStages);
-            a.next(2);
+            a.next(kAccBufs);
           }
         }
         if (T::s2 && ok) {
@@ -460,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           mma_commit(&acc_full[a.idx]);
           if (T::h_global) mma_commit(hb_free);
-          a.next(2);
+          a.next(kAccBufs);
         }
       }
       // All MMAs issued by this thread are complete before TMEM is released.
@@ -527,8 +530,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c0 = half * ncols;
 #pragma unroll
           for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+          float sx0 = row_ok ? __ldg(sx_row) : 0.0f;
+          float sx1 = (row_ok && G > 1) ? __ldg(sx_row + 1) : 0.0f;
           for (int g = 0; g < G; ++g) {
-            const float sx = row_ok ? __ldg(sx_row + g) : 0.0f;
+            const float sx = sx0;
+            sx0 = sx1;
+            sx1 = (row_ok && g + 2 < G) ? __ldg(sx_row + g + 2) : 0.0f;
             if (!(ok = wait_bar(&acc_full[a.idx], a.phase, abort_flag, kSiteDrainAccFull))) break;
             tc_fence_after();
             if (!(ok = wait_bar(&sc_full[q.idx], q.phase, abort_flag, kSiteDrainScaleFull))) break;
@@ -540,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive(&acc_empty[a.idx]);
               mbar_arrive(&sc_empty[q.idx]);
             }
-            a.next(2);
+            a.next(kAccBufs);
             q.next(kScaleSlots);
           }
           if (!ok) break;
@@ -578,8 +585,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
       if (T::res) {
+        float sx0 = row_ok ? __ldg(sx_row) : 0.0f;
+        float sx1 = (row_ok && G > 1) ? __ldg(sx_row + 1) : 0.0f;
         for (int g = 0; g < G; ++g) {
-          const float sx = row_ok ? __ldg(sx_row + g) : 0.0f;
+          const float sx = sx0;
+          sx0 = sx1;
+          sx1 = (row_ok && g + 2 < G) ? __ldg(sx_row + g + 2) : 0.0f;
           if (!(ok = wait_bar(&acc_full[a.idx], a.phase, abort_flag, kSiteDrainAccFull))) break;
           tc_fence_after();
           if (!(ok = wait_bar(&sc_full[q.idx], q.phase, abort_flag, kSiteDrainScaleFull))) break;
@@ -591,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&acc_empty[a.idx]);
             mbar_arrive(&sc_empty[q.idx]);
           }
-          a.next(2);
+          a.next(kAccBufs);
           q.next(kScaleSlots);
         }
         if (!ok) break;
@@ -655,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[a.idx]);
-        a.next(2);
+        a.next(kAccBufs);
       }
     }
   }

@@ -39,7 +39,12 @@ cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols
 cudaError_t launch_add_cast(const float* a, const float* b, int64_t count, uint16_t* y,
                             cudaStream_t stream);
 
-// Device status word (first wait site that gave up).
+// Decode-shape kernel (b <= 16, split K over a 4- or 8-CTA cluster).
+bool decode_eligible(const GemmCall& call);
+cudaError_t launch_decode(const GemmCall& call, cudaStream_t stream);
+
+// Device status words (first wait site that gave up), one per kernel family.
 cudaError_t read_and_clear_device_status(int* code);
+cudaError_t read_and_clear_decode_status(int* code);
 
 }  // namespace twq

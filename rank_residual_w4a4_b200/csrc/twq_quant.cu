@@ -4,6 +4,7 @@
 // (__fdiv_rn), round half to even (rintf).
 #include <cuda_bf16.h>
 
+#include "sm100_ptx.cuh"
 #include "twq_internal.h"
 
 namespace twq {
@@ -24,6 +25,9 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
                                                            int64_t b, int m, int64_t ldx,
                                                            uint8_t* __restrict__ xq,
                                                            float* __restrict__ sx) {
+  // The layer kernel that follows may start its prologue and weight loads now;
+  // it reads xq / sx only after this grid has completed.
+  pdl_launch_dependents();
   const int G = m / 128;
   const int pairs = (G + 1) / 2;
   const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;

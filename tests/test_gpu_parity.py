@@ -145,12 +145,58 @@ def test_variants_match_oracle(twq, device, b, m, n, r):
     _status_clean(twq)
 
 
+def _decode_path(b, m, r):
+    """Shapes the library runs on the split-K decode kernel (b <= 16, r <= 128, m <= 8192)."""
+    return 1 <= b <= 16 and r <= 128 and m // 128 <= 64
+
+
 @pytest.mark.parametrize("b,m,n,r", SHAPES)
-def test_unfused_is_bitwise_fused(twq, device, b, m, n, r):
+def test_unfused_vs_fused(twq, device, b, m, n, r):
+    """Same kernel family: bitwise equal. Decode shapes (split-K kernel for the fused
+    call): equal within the Y tolerance."""
     x, R, L1, L2 = _operands(b, m, n, r, seed=3)
     w = _pack(twq, device, R, L1, L2)
     xq, sx = twq.quantize_act(to_dev(x, device))
-    assert np.array_equal(bits_of(twq.unfused_linear(xq, sx, w)), bits_of(twq.fused_linear(xq, sx, w)))
+    yu, yf = bits_of(twq.unfused_linear(xq, sx, w)), bits_of(twq.fused_linear(xq, sx, w))
+    if _decode_path(b, m, r):
+        assert_y_close(yf, yu, "decode fused vs unfused")
+    else:
+        assert np.array_equal(yu, yf)
+    _status_clean(twq)
+
+
+DECODE_SHAPES = [  # b, m, n, r: cluster of 4 (m <= 4096) and of 8 (4096 < m <= 8192),
+    # uneven group and r-unit splits, a CTA with no groups (m = 128), r below one unit per CTA
+    (1, 4096, 512, 128), (7, 4096, 256, 128), (16, 8192, 256, 128), (16, 5120, 256, 64),
+    (5, 1024, 384, 48), (16, 128, 128, 16), (2, 640, 128, 32), (16, 4096, 128, 0),
+]
+
+
+@pytest.mark.parametrize("b,m,n,r", DECODE_SHAPES)
+def test_decode_kernel_matches_oracle(twq, device, b, m, n, r):
+    x, R, L1, L2 = _operands(b, m, n, r, seed=8)
+    w = _pack(twq, device, R, L1, L2)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    assert_y_close(bits_of(twq.fused_linear(xq, sx, w)), _oracle_y(x, R, L1, L2, oracle.FUSED),
+                   "decode fused %s" % ((b, m, n, r),))
+    assert_y_close(bits_of(twq.w4a4_only(xq, sx, w)), _oracle_y(x, R, L1, L2, oracle.W4A4_ONLY),
+                   "decode w4a4 %s" % ((b, m, n, r),))
+    if r:
+        assert_y_close(bits_of(twq.lowrank_only(xq, sx, w)),
+                       _oracle_y(x, R, L1, L2, oracle.LOWRANK_ONLY), "decode lowrank %s" % ((b, m, n, r),))
+    _status_clean(twq)
+
+
+def test_decode_identities(twq, device):
+    x, R, L1, L2 = _operands(8, 1024, 256, 64, seed=12)
+    xq, sx = twq.quantize_act(to_dev(x, device))
+    w0 = _pack(twq, device, R, None, None)
+    assert np.array_equal(bits_of(twq.fused_linear(xq, sx, w0)), bits_of(twq.w4a4_only(xq, sx, w0)))
+    wz = _pack(twq, device, np.zeros_like(R), L1, L2)
+    w = _pack(twq, device, R, L1, L2)
+    assert np.array_equal(bits_of(twq.fused_linear(xq, sx, wz)), bits_of(twq.lowrank_only(xq, sx, w)))
+    yn = bits_of(twq.w4a4_only(*twq.quantize_act(to_dev(x ^ np.uint16(0x8000), device)), w0))
+    assert np.array_equal(yn, bits_of(twq.w4a4_only(xq, sx, w0)) ^ np.uint16(0x8000))
     _status_clean(twq)
 
 

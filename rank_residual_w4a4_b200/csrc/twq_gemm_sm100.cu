@@ -17,7 +17,7 @@
 //   warp 0        TMA producer: packed 4-bit code tiles of X and R / L1, BF16
 //                 tiles of L2^T, and the per-group weight scales;
 //   warp 1        tcgen05.mma issuer (one thread) and TMEM owner;
-//   warps 4-7     unpack: 4-bit codes -> int8 in the UMMA 128-byte-swizzle
+//   warps 2-7     unpack: 4-bit codes -> int8 in the UMMA 128-byte-swizzle
 //                 K-major layout (each byte holds 16*q; the MMA result is 256x
 //                 the integer dot product and is rescaled exactly by 2^-8);
 //   warps 8-15    drain: per-group tensor-memory loads, fp32 scaling and
@@ -136,19 +136,38 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int c) {
 }
 
 // 4-bit codes (rows x 64 bytes, dense) -> int8 (rows x 128 bytes, swizzled), 16*q per byte.
+// Each thread takes 16 packed bytes (two 16-byte output chunks) per item, and
+// four items are loaded before any is stored so the shared-memory latencies
+// overlap.
 __device__ __forceinline__ void unpack_rows(const uint8_t* src, uint8_t* dst, int rows, int tid,
                                             int nthreads) {
-  const int chunks = rows * 8;
-  for (int e = tid; e < chunks; e += nthreads) {
-    const int row = e >> 3;
-    const int c = e & 7;
-    const uint2 w = *reinterpret_cast<const uint2*>(src + row * 64 + c * 8);
-    uint4 o;
-    o.x = (w.x << 4) & 0xF0F0F0F0u;
-    o.y = w.x & 0xF0F0F0F0u;
-    o.z = (w.y << 4) & 0xF0F0F0F0u;
-    o.w = w.y & 0xF0F0F0F0u;
-    *reinterpret_cast<uint4*>(dst + sw128_offset(row, c)) = o;
+  const int items = rows * 4;  // 16 packed bytes each
+  for (int e0 = tid; e0 < items; e0 += 4 * nthreads) {
+    uint4 w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = e0 + i * nthreads;
+      if (e < items) w[i] = *reinterpret_cast<const uint4*>(src + e * 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = e0 + i * nthreads;
+      if (e < items) {
+        const int row = e >> 2;
+        const int c = (e & 3) * 2;
+        uint4 o0, o1;
+        o0.x = (w[i].x << 4) & 0xF0F0F0F0u;
+        o0.y = w[i].x & 0xF0F0F0F0u;
+        o0.z = (w[i].y << 4) & 0xF0F0F0F0u;
+        o0.w = w[i].y & 0xF0F0F0F0u;
+        o1.x = (w[i].z << 4) & 0xF0F0F0F0u;
+        o1.y = w[i].z & 0xF0F0F0F0u;
+        o1.z = (w[i].w << 4) & 0xF0F0F0F0u;
+        o1.w = w[i].w & 0xF0F0F0F0u;
+        *reinterpret_cast<uint4*>(dst + sw128_offset(row, c)) = o0;
+        *reinterpret_cast<uint4*>(dst + sw128_offset(row, c + 1)) = o1;
+      }
+    }
   }
 }
 
@@ -163,30 +182,29 @@ __device__ __forceinline__ void copy_smem(const uint8_t* src, uint8_t* dst, int 
 __device__ __forceinline__ void drain_group(float (&acc)[64], uint32_t taddr, int ncols,
                                             const float* sc, float sx) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t v[32];
+  for (int h = 0; h < 4; ++h) {
+    if (h * 16 < ncols) {
+      uint32_t v[16];
+      uint32_t t0[8], t1[8];
+      tmem_ld8(taddr + h * 16, t0);
+      if (h * 16 + 8 < ncols) tmem_ld8(taddr + h * 16 + 8, t1);
+      tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < 32; c += 8)
-      if (h * 32 + c < ncols) {
-        uint32_t t[8];
-        tmem_ld8(taddr + h * 32 + c, t);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v[c + k] = t[k];
+      for (int k = 0; k < 8; ++k) {
+        v[k] = t0[k];
+        v[k + 8] = t1[k];
       }
-    tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < 32; c += 4)
-      if (h * 32 + c < ncols) {
-        const float4 s4 = *reinterpret_cast<const float4*>(sc + h * 32 + c);
-        acc[h * 32 + c + 0] =
-            fmaf(static_cast<float>(static_cast<int32_t>(v[c + 0])) * s4.x, sx, acc[h * 32 + c + 0]);
-        acc[h * 32 + c + 1] =
-            fmaf(static_cast<float>(static_cast<int32_t>(v[c + 1])) * s4.y, sx, acc[h * 32 + c + 1]);
-        acc[h * 32 + c + 2] =
-            fmaf(static_cast<float>(static_cast<int32_t>(v[c + 2])) * s4.z, sx, acc[h * 32 + c + 2]);
-        acc[h * 32 + c + 3] =
-            fmaf(static_cast<float>(static_cast<int32_t>(v[c + 3])) * s4.w, sx, acc[h * 32 + c + 3]);
-      }
+      for (int c = 0; c < 16; c += 4)
+        if (h * 16 + c < ncols) {
+          const float4 s4 = *reinterpret_cast<const float4*>(sc + h * 16 + c);
+          const int j = h * 16 + c;
+          acc[j + 0] = fmaf(static_cast<float>(static_cast<int32_t>(v[c + 0])) * s4.x, sx, acc[j + 0]);
+          acc[j + 1] = fmaf(static_cast<float>(static_cast<int32_t>(v[c + 1])) * s4.y, sx, acc[j + 1]);
+          acc[j + 2] = fmaf(static_cast<float>(static_cast<int32_t>(v[c + 2])) * s4.z, sx, acc[j + 2]);
+          acc[j + 3] = fmaf(static_cast<float>(static_cast<int32_t>(v[c + 3])) * s4.w, sx, acc[j + 3]);
+        }
+    }
   }
 }
 
@@ -248,10 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPackedStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 4);
+      mbar_init(&empty[i], 6);
     }
     for (int i = 0; i < kUnpackedStages; ++i) {
-      mbar_init(&ufull[i], 4);
+      mbar_init(&ufull[i], 6);
       mbar_init(&uempty[i], 1);
     }
     for (int i = 0; i < kAccBufs; ++i) {
@@ -471,9 +489,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int dummy = 0;
       wait_bar(mma_done, 0, &dummy, kSiteFinal);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 2 && warp < 8) {
     // --------------------------------------------------------------- unpack
-    const int tid = threadIdx.x - 128;
+    const int tid = threadIdx.x - 64;
     Ring s, u;
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t) {
@@ -492,10 +510,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int hc = step / G;
             brows = min(kHChunk, args.r - hc * kHChunk);
           }
-          unpack_rows(src, dst, kBM, tid, 128);
-          unpack_rows(src + L::kSlotA, dst + L::kUA, brows, tid, 128);
+          unpack_rows(src, dst, kBM, tid, 192);
+          unpack_rows(src + L::kSlotA, dst + L::kUA, brows, tid, 192);
         } else {
-          copy_smem(src, dst + L::kUA, BN * 128, tid, 128);
+          copy_smem(src, dst + L::kUA, BN * 128, tid, 192);
         }
         fence_proxy_async_smem();
         __syncwarp();

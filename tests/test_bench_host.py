@@ -1,0 +1,67 @@
+"""Host logic of bench.py: byte and op counts, roofline entries, the traffic table, and the
+max-over-ranks reduction across two processes (gloo, CPU)."""
+import os
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+from rank_residual_w4a4_b200 import _build, twq
+
+
+def test_weight_bytes_match_the_abi_size_query():
+    _build.build()
+    for m, n, r in ((512, 512, 32), (4096, 4096, 128), (14336, 4096, 256), (5120, 25600, 0)):
+        assert bench.weight_bytes(m, n, r) == sum(twq.weights_sizes(m, n, r))
+        b = 16
+        xq, sx = twq.act_sizes(b, m)
+        assert bench.act_bytes(b, m, n) == xq + sx + 2 * b * n
+
+
+def test_op_counts():
+    assert bench.int8_ops(2048, 4096, 14336, 128) == 2 * 2048 * 4096 * 14336 + 2 * 2048 * 4096 * 128
+    assert bench.bf16_flops(2048, 14336, 128) == 2 * 2048 * 128 * 14336
+
+
+def test_roofline_entries():
+    peaks = (6453.7, 1686.7, 1412.9, "measured")
+    d = bench.roofline_entry("decode16", 13.3e-6, peaks, None)
+    assert d["bound"] == "hbm" and d["unit"] == "GB/s"
+    assert abs(d["achieved"] - d["algorithmic_bytes"] / 13.3e-6 / 1e9) < 0.1
+    assert abs(d["frac"] - d["achieved"] / 6453.7) < 1e-4
+    p = bench.roofline_entry("gateup", 500e-6, peaks, 123)
+    assert p["bound"] == "tensor" and p["peak"] == round(1686.7 * 2, 1) and p["traffic"] == 123
+
+
+def test_traffic_table_is_tied_to_the_kernel_sources():
+    h = bench.kernel_source_hash()
+    path = os.path.join(bench.ROOT, "profiles", "fused_kernel_traffic.txt")
+    lines = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    for wl, nbytes, hh in lines:
+        got = bench.profiled_traffic(wl)
+        assert got == (int(nbytes) if hh == h else None)
+
+
+def _rank_main(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    v = bench.max_over_ranks(1.0 + rank, world, torch.device("cpu"))
+    bench.barrier(world)
+    out[rank] = v
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_processes():
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert dict(out) == {0: 2.0, 1: 2.0}

@@ -3,9 +3,12 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl twq|reference]
 
-One step is one pass of the hot path over one batch: the online activation
-quantizer (twq_quantize_act) and the fused dual-component layer
-(twq_fused_linear) on inputs already resident in HBM. Steps run from a CUDA
+One step is one pass of the hot path over one batch on inputs already resident
+in HBM: BF16 X to BF16 Y through the online activation quantizer and the fused
+dual-component layer. For decode batches (b <= 16) that is one launch of
+twq_fused_linear_x, which quantizes X inside the layer kernel; otherwise it is
+twq_quantize_act followed by twq_fused_linear (the two-call step is timed for
+decode batches too and reported beside it). Steps run from a CUDA
 graph on one stream; the K timed steps are bracketed by a barrier and a device
 synchronize, timed with CUDA events, max over ranks. Packed weights rotate over
 enough copies that consecutive uses of one copy are more than 2x the 126 MB L2
@@ -59,8 +62,11 @@ def weight_bytes(m, n, r):
     return m * n // 2 + 4 * (m // 128) * n + m * r // 2 + 4 * (m // 128) * r + 2 * r * n
 
 
-def act_bytes(b, m, n):
-    return b * m // 2 + 4 * b * (m // 128) + 2 * b * n
+def act_bytes(b, m, n, bf16_x=False):
+    """Activation bytes of one layer call: X in (codes and scales, or BF16 X for the
+    kernel that quantizes it itself) and BF16 Y out."""
+    x_in = 2 * b * m if bf16_x else b * m // 2 + 4 * b * (m // 128)
+    return x_in + 2 * b * n
 
 
 def int8_ops(b, m, n, r):
@@ -243,16 +249,27 @@ class Problem:
         self.y = [torch.empty((b, self.n), dtype=torch.bfloat16, device=device) for _ in range(copies)]
         del R, L1, L2
 
-    def step(self, i, fused=True, ev=None):
+    @property
+    def one_launch(self):
+        """Decode batches: the layer kernel quantizes X itself (twq_fused_linear_x)."""
+        return 1 <= self.b <= 16 and (self.r == 0 or self.r <= 128) and self.m <= 8192
+
+    def step(self, i):
+        if self.one_launch:
+            self.step_x(i)
+        else:
+            self.step_two_call(i)
+
+    def step_x(self, i):
+        from rank_residual_w4a4_b200 import twq
+        c = i % self.copies
+        twq.fused_linear_x(self.x[c], self.weights[c], self.y[c])
+
+    def step_two_call(self, i):
         from rank_residual_w4a4_b200 import twq
         c = i % self.copies
         twq.quantize_act(self.x[c], self.xq[c], self.sx[c])
-        if ev is not None:
-            ev[0].record()
-        if fused:
-            twq.fused_linear(self.xq[c], self.sx[c], self.weights[c], self.y[c])
-        if ev is not None:
-            ev[1].record()
+        twq.fused_linear(self.xq[c], self.sx[c], self.weights[c], self.y[c])
 
 
 def capture(fn, count):
@@ -294,12 +311,12 @@ def kernel_only_time(prob, fn, steps, reps=1):
     return s.elapsed_time(e) / 1e3 / (steps * reps)
 
 
-def roofline_entry(name, t_kernel, peaks, traffic):
+def roofline_entry(name, t_kernel, peaks, traffic, bf16_x=False):
     wl, b = describe(name)
     hbm, bf16, bf16_sus, src = peaks
     m, n, r = wl.m, wl.n, wl.r
     if b <= 64:  # decode shapes: HBM-bound
-        alg = weight_bytes(m, n, r) + act_bytes(b, m, n)
+        alg = weight_bytes(m, n, r) + act_bytes(b, m, n, bf16_x)
         ach = alg / t_kernel / 1e9
         return {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(ach / hbm, 4), "traffic": traffic,
@@ -353,13 +370,15 @@ def run_gpu(args):
     elapsed = time_graph(gk, world, device)
     t_load1 = time.time()
     elapsed = max_over_ranks(elapsed, world, device)
-    # the fused kernel alone: CUDA events around a graph of K back-to-back launches
+    # the layer kernel alone: CUDA events around a graph of K back-to-back launches
     # on the same stream and weight rotation (no events between launches, which
     # would serialize them)
     def fused_only(i):
         c = i % prob.copies
         twq.fused_linear(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c])
-    t_fused = kernel_only_time(prob, fused_only, K)
+    one = prob.one_launch
+    t_fused = kernel_only_time(prob, prob.step_x if one else fused_only, K)
+    t_two = time_graph(capture(prob.step_two_call, K), world, device) / K if one else None
     st = twq.device_status()
     if st != 0:
         raise RuntimeError("device wait timed out at site %d" % st)
@@ -387,19 +406,24 @@ def run_gpu(args):
         "data": "synthetic (seeded generator; no dataset or trained weights)",
         "config": {"workload": "%s: b=%d m=%d n=%d r=%d, group 128" % (name, b, wl.m, wl.n, wl.r),
                    "b": b, "m": wl.m, "n": wl.n, "r": wl.r, "parallelism": "replicas x%d" % world,
-                   "step": "twq_quantize_act + twq_fused_linear",
+                   "step": ("twq_fused_linear_x (activation quantizer inside the layer kernel)"
+                            if one else "twq_quantize_act + twq_fused_linear"),
                    "l2": "weights rotate over %d copies (%.0f MB > 2x L2)" % (
                        prob.copies, prob.copies * weight_bytes(wl.m, wl.n, wl.r) / 1e6),
                    "launch": "CUDA graph of the K timed steps; the fused kernel is "
                              "launched with programmatic stream serialization"},
         "effective_tops": round(ops * world * K / elapsed / 1e12, 3),
         "fused_kernel_us": round(t_fused * 1e6, 3),
-        "fused_kernel_timing": "events around a graph of K back-to-back fused launches",
-        "roofline": roofline_entry(name, t_fused, peaks, profiled_traffic(name)),
+        "fused_kernel_timing": "events around a graph of K back-to-back layer launches",
+        "roofline": roofline_entry(name, t_fused, peaks,
+                                   profiled_traffic(name + ("_x" if one else "")), bf16_x=one),
         "e2e": e2e,
-        "gpu_launches": 2 * K,
+        "gpu_launches": (1 if one else 2) * K,
         "clocks": clk,
     }
+    if one:
+        line["two_call_step_us"] = round(t_two * 1e6, 3)
+        line["two_call_step"] = "twq_quantize_act + twq_fused_linear, same graph timing"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(name, seconds=args.cpu_seconds)
     if rank == 0 and world == 1 and not args.no_sweep:
@@ -414,7 +438,7 @@ def run_gpu(args):
 
 def run_e2e(prob, K, W, world, device):
     """Same metric through the Python binding with host buffers: per step an H2D copy of
-    X from pinned memory, quantize + fused layer, and a D2H copy of Y."""
+    X from pinned memory, the layer step of run_gpu, and a D2H copy of Y."""
     import torch
     from rank_residual_w4a4_b200 import twq
     xh = torch.from_numpy(prob.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -424,8 +448,11 @@ def run_e2e(prob, K, W, world, device):
     def one(i):
         c = i % prob.copies
         xd.copy_(xh, non_blocking=True)
-        xq, sx = twq.quantize_act(xd, prob.xq[c], prob.sx[c])
-        y = twq.fused_linear(xq, sx, prob.weights[c], prob.y[c])
+        if prob.one_launch:
+            y = twq.fused_linear_x(xd, prob.weights[c], prob.y[c])
+        else:
+            xq, sx = twq.quantize_act(xd, prob.xq[c], prob.sx[c])
+            y = twq.fused_linear(xq, sx, prob.weights[c], prob.y[c])
         yh.copy_(y, non_blocking=True)
 
     for i in range(W):
@@ -475,6 +502,7 @@ def sweep(args, device, peaks):
             c = i % prob.copies
             twq.quantize_act(prob.x[c], prob.xq[c], prob.sx[c])
 
+
         for i in range(prob.copies):
             quant(i)
         torch.cuda.synchronize()
@@ -482,6 +510,7 @@ def sweep(args, device, peaks):
         t_w = kernel_only_time(prob, w4, steps, reps=3)
         t_u = kernel_only_time(prob, unf, steps, reps=3)
         t_q = kernel_only_time(prob, quant, steps, reps=3)
+        t_x = kernel_only_time(prob, prob.step_x, steps, reps=3) if prob.one_launch else None
         ops = int8_ops(b, wl.m, wl.n, wl.r) + bf16_flops(b, wl.n, wl.r)
         res.update({
             "fused_us": round(t_f * 1e6, 2), "w4a4_only_us": round(t_w * 1e6, 2),
@@ -491,6 +520,11 @@ def sweep(args, device, peaks):
             "roofline": roofline_entry(name, t_f, peaks, profiled_traffic(name)),
             "timing": "graph of back-to-back launches, weights rotating over %d copies" % prob.copies,
         })
+        if t_x is not None:
+            res["fused_x_us"] = round(t_x * 1e6, 2)
+            res["tokens_per_s"] = round(b / t_x, 1)
+            res["roofline_x"] = roofline_entry(name, t_x, peaks, profiled_traffic(name + "_x"),
+                                               bf16_x=True)
         out.append(res)
         del prob, ws
         torch.cuda.empty_cache()

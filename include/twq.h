@@ -141,6 +141,24 @@ TWQ_API twq_status twq_pack_weights(const uint16_t* R, const uint16_t* L1, const
 TWQ_API twq_status twq_fused_linear(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
                             uint16_t* y, twq_stream_t stream);
 
+/*
+ * The fused layer with the activation quantizer inside it, for decode batches
+ * (TwinQuant §4.3: the activation is quantized once, on chip, and the codes feed
+ * both the residual GEMM and the first low-rank GEMM). Each CTA quantizes its
+ * slice of X straight into shared memory, so Q(X) never goes to HBM and the
+ * whole layer is one launch.
+ *   x    b x m BF16, row stride ldx elements (ldx >= m, ldx % 8 == 0), finite
+ *   w    from twq_pack_weights;  y  b x n BF16 (output)
+ * Result: bitwise identical to twq_quantize_act followed by twq_fused_linear.
+ * Limits: 1 <= b <= 16, m <= 8192, r <= 128 (b == 0 is a no-op); other shapes
+ * return TWQ_ERR_UNSUPPORTED and launch nothing (use the two-call path).
+ * Launched with programmatic stream serialization like twq_fused_linear: X may
+ * come from the preceding kernel; the weights must not be written by a kernel
+ * that signals early.
+ */
+TWQ_API twq_status twq_fused_linear_x(const uint16_t* x, int64_t ldx, int64_t b,
+                                      const twq_weights* w, uint16_t* y, twq_stream_t stream);
+
 /* Residual component only: Y = bf16(Q(X) Q(R)) (TwinQuant Eq. (2)); ignores l1q/sl1/l2t. */
 TWQ_API twq_status twq_w4a4_only(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
                          uint16_t* y, twq_stream_t stream);

@@ -146,6 +146,28 @@ twq_status twq_lowrank_only(const uint8_t* xq, const float* sx, int64_t b, const
   return run(twq::kModeLowRank, xq, sx, b, w, y, nullptr, stream);
 }
 
+twq_status twq_fused_linear_x(const uint16_t* x, int64_t ldx, int64_t b, const twq_weights* w,
+                              uint16_t* y, twq_stream_t stream) {
+  if (!w) return TWQ_ERR_INVALID_ARG;
+  twq_status s = shape_ok(w->m, w->n, w->r);
+  if (s != TWQ_OK) return s;
+  if (b < 0 || ldx < w->m) return TWQ_ERR_INVALID_ARG;
+  if (b == 0) return TWQ_OK;
+  if (!x || !y || !w->rq || !w->sr) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || ldx % 8 || !aligned16(y) || !aligned16(w->rq) || !aligned16(w->sr))
+    return TWQ_ERR_MISALIGNED;
+  const bool lr = w->r > 0;
+  if (lr) {
+    if (!w->l1q || !w->sl1 || !w->l2t) return TWQ_ERR_INVALID_ARG;
+    if (!aligned16(w->l1q) || !aligned16(w->sl1) || !aligned16(w->l2t)) return TWQ_ERR_MISALIGNED;
+  }
+  twq::GemmCall c{lr ? twq::kModeFused : twq::kModeW4A4, nullptr, nullptr, b, w, y, nullptr};
+  c.x = x;
+  c.ldx = ldx;
+  if (!twq::decode_eligible(c)) return TWQ_ERR_UNSUPPORTED;
+  return from_cuda(twq::launch_decode(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t twq_unfused_workspace_bytes(int64_t b, int64_t n, int64_t r) {
   if (b <= 0 || n <= 0 || r < 0) return 0;
   // Y_res fp32 (b x n) | Y_lr fp32 (b x n) | H bf16 (b x r), each 256-byte aligned
@@ -193,9 +215,9 @@ int twq_launches_per_call(const char* ep) {
   if (!strcmp(ep, "twq_quantize_act")) return 1;
   if (!strcmp(ep, "twq_pack_weights")) return 3;
   if (!strcmp(ep, "twq_fused_linear") || !strcmp(ep, "twq_w4a4_only") ||
-      !strcmp(ep, "twq_lowrank_only"))
+      !strcmp(ep, "twq_lowrank_only") || !strcmp(ep, "twq_fused_linear_x"))
     return 1;
-  if (!strcmp(ep, "twq_unfused_linear")) return 4;
+  if (!strcmp(ep, "twq_unfused_linear") || !strcmp(ep, "twq_unfused_linear_noalloc")) return 4;
   return -1;
 }
 

@@ -30,6 +30,7 @@
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
+#include "twq_eq1.cuh"
 #include "twq_internal.h"
 
 namespace twq {
@@ -78,8 +79,9 @@ struct DLayout {
   static constexpr int kOffXu = kOffL1 + kMaxGroups * 8192;    // kMaxGroups x 2 KB (SW128)
   static constexpr int kOffL2 = kOffXu + kMaxGroups * 2048;    // 16 KB (SW128)
   static constexpr int kOffHb = kOffL2 + 16384;                // 2 KB (SW128)
-  static constexpr int kOffXp = kOffHb + 2048;                 // kMaxGroups x 1 KB
-  static constexpr int kOffSx = kOffXp + kMaxGroups * 1024;    // [group][token] fp32
+  static constexpr int kOffXp = kOffHb + 2048;                 // kMaxGroups x 1 KB codes, or
+                                                               // kMaxGroups x 4 KB BF16 X
+  static constexpr int kOffSx = kOffXp + kMaxGroups * 4096;    // [group][token] fp32
   static constexpr int kOffHred = kOffSx + kMaxGroups * kNT * 4;
   static constexpr int kHredBytes = 128 * kNT * 4;             // [src][c][t], KS * slice <= 128
   static constexpr int kOffYred = kOffHred + kHredBytes;
@@ -145,13 +147,64 @@ __device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int j, uin
   tmem_st32(taddr, v);
 }
 
+// Eq. (1) quantizer fused into the prologue. The CTA's BF16 slice of X sits in
+// shared memory as two TMA boxes per group (64 elements x 16 tokens each, rows
+// of 128 bytes; tokens >= b read as zero). Half-warp `hw` of the 20 turns the
+// (token, group) pairs hw, hw + 20, ... into int8 codes (16*q, in the in-chunk
+// order of unpack8) in the 128-byte-swizzle B tiles and fp32 scales in sxs,
+// with the arithmetic of twq_quantize_act, so the codes are identical.
+constexpr int kQHalfWarps = 20;  // quantizing half-warps: warps 2-3 and 12-19
+
+__device__ __forceinline__ void quantize_slice(const uint8_t* xs, int ng, uint8_t* xu, float* sxs,
+                                               int hw, int lane) {
+  const int l = lane & 15;
+  const int pairs = kNT * ng;
+  const int iters = (pairs + kQHalfWarps - 1) / kQHalfWarps;  // the same for both halves of a warp
+#pragma unroll 1
+  for (int it = 0; it < iters; ++it) {
+    const int p = hw + it * kQHalfWarps;
+    const bool pv = p < pairs;
+    const int gi = pv ? p / kNT : 0, t = pv ? p % kNT : 0;
+    const uint4 raw = *reinterpret_cast<const uint4*>(xs + gi * 4096 + (l >> 3) * 2048 + t * 128 +
+                                                      (l & 7) * 16);
+    float f[8];
+    f[0] = __uint_as_float(raw.x << 16);
+    f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(raw.y << 16);
+    f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    f[4] = __uint_as_float(raw.z << 16);
+    f[5] = __uint_as_float(raw.z & 0xFFFF0000u);
+    f[6] = __uint_as_float(raw.w << 16);
+    f[7] = __uint_as_float(raw.w & 0xFFFF0000u);
+    float a = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(f[k]));
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+    const Eq1Scale ks = eq1_scale(a);
+    uint32_t w0 = 0, w1 = 0;
+    if (ks.s != 0.0f) {
+      float c[8];
+      eq1_codes8(f, ks, c);
+      w0 = (eq1_nibble(c[0]) << 4) | (eq1_nibble(c[2]) << 12) | (eq1_nibble(c[4]) << 20) |
+           (eq1_nibble(c[6]) << 28);
+      w1 = (eq1_nibble(c[1]) << 4) | (eq1_nibble(c[3]) << 12) | (eq1_nibble(c[5]) << 20) |
+           (eq1_nibble(c[7]) << 28);
+    }
+    if (pv) {
+      *reinterpret_cast<uint2*>(xu + gi * 2048 + d_sw128(t, l >> 1) + (l & 1) * 8) = make_uint2(w0, w1);
+      if (l == 0) sxs[gi * kNT + t] = ks.s;
+    }
+  }
+}
+
 // Range of 16-column units of r owned by cluster rank k.
 __device__ __forceinline__ void unit_range(int U, int KS, int k, int& u0, int& u1) {
   u0 = k * U / KS;
   u1 = (k + 1) * U / KS;
 }
 
-template <int kMode, int KS>
+template <int kMode, int KS, bool kQ>
 __global__ void __launch_bounds__(kThreads, 1)
     twq_decode_kernel(const __grid_constant__ CUtensorMap tm_rq,
                       const __grid_constant__ CUtensorMap tm_l1q,
@@ -227,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 31) {
       mbar_init(xfull, 1);
-      mbar_init(xready, 2);
+      mbar_init(xready, kQ ? 10 : 2);
       mbar_init(l2full, 1);
       mbar_init(hb_ready, 4);
       mbar_init(lr_full, 1);
@@ -263,11 +316,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(l2full, 16384);
         tma_load_2d(l2s, &tm_l2t, l2full, u0 * 16, n0);
       }
-      // The activation codes may come from the kernel just before this one on the
+      // The activations may come from the kernel just before this one on the
       // stream (launched with programmatic serialization): wait for it first.
       pdl_wait();
-      mbar_arrive_expect_tx(xfull, ng * 1024);
-      for (int gi = 0; gi < ng; ++gi) tma_load_2d(xp + gi * 1024, &tm_xq, xfull, (g0 + gi) * 64, 0);
+      if (kQ) {  // BF16 X: two boxes of 64 elements x 16 tokens per group
+        mbar_arrive_expect_tx(xfull, ng * 4096);
+        for (int gi = 0; gi < ng; ++gi) {
+          tma_load_2d(xp + gi * 4096, &tm_xq, xfull, (g0 + gi) * 128, 0);
+          tma_load_2d(xp + gi * 4096 + 2048, &tm_xq, xfull, (g0 + gi) * 128 + 64, 0);
+        }
+      } else {
+        mbar_arrive_expect_tx(xfull, ng * 1024);
+        for (int gi = 0; gi < ng; ++gi) tma_load_2d(xp + gi * 1024, &tm_xq, xfull, (g0 + gi) * 64, 0);
+      }
     }
   }
   if (warp == 1) {
@@ -282,6 +343,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
+  if (kQ && (warp == 2 || warp == 3 || warp >= 12)) {
+    // ----- X quantize (warps 2-3 and 12-19; 12-19 then go on to their own roles)
+    const int hw = (warp < 4 ? warp - 2 : warp - 10) * 2 + (lane >> 4);
+    if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) {
+      quantize_slice(xp, ng, xu, sxs, hw, lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xready);
+    }
+  }
   if (warp == 0) {
     // ------------------------------------ residual MMA issuer (lane 0 of warp 0)
     if (lane == 0) {
@@ -352,31 +423,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       d_wait<false>(mma_done, 0, &never, kDSiteFinal);
     }
   } else if (warp < 4) {
-    // ------------------------------------------------ X unpack (warps 2 and 3)
-    const int tid = threadIdx.x - 64;
-    pdl_wait();    // the scales, like the codes, may come from the preceding kernel
-    float sxv[2];  // activation scales, loaded before the codes arrive
+    // the quantizing variant did its X work above; warps 2-3 have no other role
+    if constexpr (!kQ) {
+      // ------------------------------------------------ X unpack (warps 2 and 3)
+      const int tid = threadIdx.x - 64;
+      pdl_wait();    // the scales, like the codes, may come from the preceding kernel
+      float sxv[2];  // activation scales, loaded before the codes arrive
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int e = tid + 64 * i;
-      const int gi = e / kNT, t = e % kNT;
-      sxv[i] = (gi < ng && t < args.b) ? __ldg(args.sx + static_cast<int64_t>(t) * G + g0 + gi) : 0.0f;
-    }
-    if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) {
-      for (int e = tid; e < ng * kNT * 8; e += 64) {
-        const int gi = e / (kNT * 8);
-        const int row = (e / 8) % kNT;
-        const int c = e & 7;
-        const uint2 w = *reinterpret_cast<const uint2*>(xp + gi * 1024 + row * 64 + c * 8);
-        uint32_t o[4];
-        unpack8(w.x, w.y, o);
-        *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(row, c)) = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int i = 0; i < 2; ++i) {
+        const int e = tid + 64 * i;
+        const int gi = e / kNT, t = e % kNT;
+        sxv[i] = (gi < ng && t < args.b) ? __ldg(args.sx + static_cast<int64_t>(t) * G + g0 + gi) : 0.0f;
       }
+      if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) {
+        for (int e = tid; e < ng * kNT * 8; e += 64) {
+          const int gi = e / (kNT * 8);
+          const int row = (e / 8) % kNT;
+          const int c = e & 7;
+          const uint2 w = *reinterpret_cast<const uint2*>(xp + gi * 1024 + row * 64 + c * 8);
+          uint32_t o[4];
+          unpack8(w.x, w.y, o);
+          *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(row, c)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
 #pragma unroll
-      for (int i = 0; i < 2; ++i) sxs[tid + 64 * i] = sxv[i];
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xready);
+        for (int i = 0; i < 2; ++i) sxs[tid + 64 * i] = sxv[i];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xready);
+      }
     }
   } else if (warp < 12) {
     // -------- operand tiles -> tensor memory: L1 (warps 4-7) and R (warps 8-11)
@@ -539,7 +613,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -579,7 +652,7 @@ bool d_encode(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int kMode, int KS>
+template <int kMode, int KS, bool kQ>
 cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
   const twq_weights* w = c.w;
   DecodeArgs a{};
@@ -594,8 +667,10 @@ cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
   a.G = a.m / 128;
   CUtensorMap m_rq{}, m_l1q{}, m_xq{}, m_l2t{};
   const uint64_t kb = static_cast<uint64_t>(a.m / 2);
-  bool ok = d_encode(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, kb, c.b, kb, 64, kNT,
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
+  bool ok = kQ ? d_encode(&m_xq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.x, a.m, c.b,
+                          static_cast<uint64_t>(c.ldx) * 2, 64, kNT, CU_TENSOR_MAP_SWIZZLE_NONE)
+                : d_encode(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, kb, c.b, kb, 64, kNT,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
   if (DTraits<kMode>::res)
     ok = ok && d_encode(&m_rq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->rq, kb, a.n, kb, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_64B);
@@ -606,7 +681,7 @@ cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
     ok = ok && d_encode(&m_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2t, a.r, a.n,
                         static_cast<uint64_t>(a.r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
-  auto kern = twq_decode_kernel<kMode, KS>;
+  auto kern = twq_decode_kernel<kMode, KS, kQ>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DLayout::kAlloc);
   if (e != cudaSuccess) return e;
@@ -646,17 +721,19 @@ bool decode_eligible(const GemmCall& c) {
 cudaError_t launch_decode(const GemmCall& c, cudaStream_t st) {
   const int64_t G = c.w->m / 128;
   const bool ks8 = G > 4 * kMaxGroups;
+  const bool q = c.x != nullptr;
+#define TWQ_DECODE_CASE(MODE)                                                         \
+  if (q) return ks8 ? launch_decode_mode<MODE, 8, true>(c, st)                       \
+                    : launch_decode_mode<MODE, 4, true>(c, st);                      \
+  return ks8 ? launch_decode_mode<MODE, 8, false>(c, st) : launch_decode_mode<MODE, 4, false>(c, st);
   switch (c.mode) {
-    case kModeFused:
-      return ks8 ? launch_decode_mode<kModeFused, 8>(c, st) : launch_decode_mode<kModeFused, 4>(c, st);
-    case kModeW4A4:
-      return ks8 ? launch_decode_mode<kModeW4A4, 8>(c, st) : launch_decode_mode<kModeW4A4, 4>(c, st);
-    case kModeLowRank:
-      return ks8 ? launch_decode_mode<kModeLowRank, 8>(c, st)
-                 : launch_decode_mode<kModeLowRank, 4>(c, st);
+    case kModeFused: { TWQ_DECODE_CASE(kModeFused) }
+    case kModeW4A4: { TWQ_DECODE_CASE(kModeW4A4) }
+    case kModeLowRank: { TWQ_DECODE_CASE(kModeLowRank) }
     default:
       return cudaErrorInvalidValue;
   }
+#undef TWQ_DECODE_CASE
 }
 
 cudaError_t read_and_clear_decode_status(int* code) {

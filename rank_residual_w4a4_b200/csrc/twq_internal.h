@@ -26,6 +26,8 @@ struct GemmCall {
   const twq_weights* w;
   void* out;                // bf16 Y, fp32 b x n, or bf16 H (b x r)
   const uint16_t* h_global; // kModeS2F32 only: bf16 H, b x r
+  const uint16_t* x = nullptr;  // decode kernel only: BF16 X, quantized in the kernel
+  int64_t ldx = 0;
 };
 
 // Host-side launchers; all return cudaSuccess or the launch error.

@@ -1,10 +1,11 @@
 // Quantization and packing kernels (TwinQuant §2, Eq. (1), groups of 128 along
 // the reduction dimension per §5.1). HBM-bound: 128-bit loads, warp-shuffle
-// absmax, one correctly rounded fp32 division per scale and per element
-// (__fdiv_rn), round half to even (rintf).
+// absmax, a correctly rounded scale per group, and per element the code of the
+// correctly rounded quotient, round half to even (twq_eq1.cuh).
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
+#include "twq_eq1.cuh"
 #include "twq_internal.h"
 
 namespace twq {
@@ -12,12 +13,6 @@ namespace {
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
 
-// Eq. (1) code of v for scale s (s > 0), q_max = 7, as a 4-bit two's-complement nibble.
-__device__ __forceinline__ uint32_t code_nibble(float v, float s) {
-  float t = rintf(__fdiv_rn(v, s));
-  t = fminf(fmaxf(t, -7.0f), 7.0f);
-  return static_cast<uint32_t>(static_cast<int32_t>(t)) & 0xFu;
-}
 
 // One half-warp per (token, group): lane l of the half covers elements
 // [8l, 8l + 8) of the group; a warp covers two consecutive groups of one row.
@@ -53,11 +48,14 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
   for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(f[k]));
 #pragma unroll
   for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-  const float s = __fdiv_rn(a, 7.0f);
+  const Eq1Scale ks = eq1_scale(a);
+  const float s = ks.s;
   uint32_t word = 0;
   if (s != 0.0f) {
+    float t[8];
+    eq1_codes8(f, ks, t);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) word |= code_nibble(f[k], s) << (4 * k);
+    for (int k = 0; k < 8; ++k) word |= eq1_nibble(t[k]) << (4 * k);
   }
   if (valid) {
     *reinterpret_cast<uint32_t*>(xq + row * (m / 2) + g * 64 + l * 4) = word;
@@ -76,7 +74,8 @@ __global__ void __launch_bounds__(128) pack_cols_kernel(const uint16_t* __restri
   const uint16_t* p = w + static_cast<int64_t>(g) * 128 * cols + j;
   float a = 0.0f;
   for (int k = 0; k < 128; ++k) a = fmaxf(a, fabsf(bf16_bits_to_f32(__ldg(p + static_cast<int64_t>(k) * cols))));
-  const float sc = __fdiv_rn(a, 7.0f);
+  const Eq1Scale ks = eq1_scale(a);
+  const float sc = ks.s;
   s[static_cast<int64_t>(g) * cols + j] = sc;
   uint4* dst = reinterpret_cast<uint4*>(q + static_cast<int64_t>(j) * (m / 2) + g * 64);
 #pragma unroll 1
@@ -86,12 +85,13 @@ __global__ void __launch_bounds__(128) pack_cols_kernel(const uint16_t* __restri
     for (int wi = 0; wi < 4; ++wi) {
       uint32_t word = 0;
       if (sc != 0.0f) {
+        float v[8], t[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int kk = c * 32 + wi * 8 + k;
-          word |= code_nibble(bf16_bits_to_f32(__ldg(p + static_cast<int64_t>(kk) * cols)), sc)
-                  << (4 * k);
-        }
+        for (int k = 0; k < 8; ++k)
+          v[k] = bf16_bits_to_f32(__ldg(p + static_cast<int64_t>(c * 32 + wi * 8 + k) * cols));
+        eq1_codes8(v, ks, t);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) word |= eq1_nibble(t[k]) << (4 * k);
       }
       words[wi] = word;
     }

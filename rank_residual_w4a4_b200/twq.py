@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "TWQ_OK", 1: "TWQ_ERR_INVALID_ARG", 2: "TWQ_ERR_UNSUPPORTED",
 EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_sizes",
            "twq_quantize_act", "twq_pack_weights", "twq_fused_linear", "twq_w4a4_only",
            "twq_lowrank_only", "twq_unfused_workspace_bytes", "twq_unfused_linear",
-           "twq_device_status", "twq_launches_per_call", "twq_unfused_linear_noalloc")
+           "twq_device_status", "twq_launches_per_call", "twq_unfused_linear_noalloc",
+           "twq_fused_linear_x")
 
 
 class TwqError(RuntimeError):
@@ -69,6 +70,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twq_device_status": ([P], ctypes.c_int),
         "twq_launches_per_call": ([ctypes.c_char_p], ctypes.c_int),
         "twq_unfused_linear_noalloc": ([P, P, I, P, P, P], ctypes.c_int),
+        "twq_fused_linear_x": ([P, I, I, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -184,6 +186,28 @@ def _layer(fn: str, xq, sx, w: Weights, y, stream):
 
 def fused_linear(xq, sx, w: Weights, y=None, stream=None):
     return _layer("twq_fused_linear", xq, sx, w, y, stream)
+
+
+def fused_linear_x(x: torch.Tensor, w: Weights, y=None, stream=None):
+    """BF16 X (b x m, rows may be strided) -> Y in one launch, quantizing X inside
+    the layer kernel (decode batches, b <= 16)."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise TypeError("x must be a 2-D torch tensor")
+    if not x.is_cuda:
+        raise ValueError("x must be on a CUDA device (the library has no CPU path)")
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be torch.bfloat16, got %s" % x.dtype)
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along m")
+    b = x.shape[0]
+    ldx = x.stride(0) if b > 1 else x.shape[1]
+    if y is None:
+        y = torch.empty((b, w.n), dtype=torch.bfloat16, device=x.device)
+    cw = w.c_struct()
+    _check(load().twq_fused_linear_x(x.data_ptr(), ldx, b, ctypes.byref(cw),
+                                     _dev(y, "y", torch.bfloat16), _stream(stream)),
+           "twq_fused_linear_x")
+    return y
 
 
 def w4a4_only(xq, sx, w: Weights, y=None, stream=None):

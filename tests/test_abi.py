@@ -106,6 +106,25 @@ def test_layer_validation(lib, fn):
         assert f(A, A, 4, ctypes.byref(misw), A, None) == 3
 
 
+def test_fused_linear_x_validation(lib):
+    f = lib.twq_fused_linear_x
+    w = _w()
+    assert f(None, 512, 4, ctypes.byref(w), A, None) == 1
+    assert f(A, 512, 4, None, A, None) == 1
+    assert f(A, 256, 4, ctypes.byref(w), A, None) == 1       # ldx < m
+    assert f(A, 512, -1, ctypes.byref(w), A, None) == 1
+    assert f(A + 2, 512, 4, ctypes.byref(w), A, None) == 3
+    assert f(A, 516, 4, ctypes.byref(w), A, None) == 3       # row stride breaks 16 bytes
+    assert f(A, 512, 4, ctypes.byref(w), A + 4, None) == 3
+    assert f(A, 512, 0, ctypes.byref(w), None, None) == 0    # b == 0: nothing to do
+    # outside the in-kernel quantizer's limits: rejected, nothing launched
+    assert f(A, 512, 17, ctypes.byref(w), A, None) == 2      # b > 16
+    assert f(A, 512, 4, ctypes.byref(_w(r=144)), A, None) == 2
+    assert f(A, 8320, 4, ctypes.byref(_w(m=8320)), A, None) == 2  # m/128 > 64
+    big = _w(r=272)
+    assert f(A, 512, 4, ctypes.byref(big), A, None) == 2
+
+
 def test_lowrank_needs_rank(lib):
     w = _w(r=0)
     assert lib.twq_lowrank_only(A, A, 4, ctypes.byref(w), A, None) == 1
@@ -131,6 +150,8 @@ def test_pack_validation(lib):
 def test_launch_accounting(lib):
     assert twq.launches_per_call("twq_fused_linear") == 1
     assert twq.launches_per_call("twq_unfused_linear") == 4
+    assert twq.launches_per_call("twq_unfused_linear_noalloc") == 4
+    assert twq.launches_per_call("twq_fused_linear_x") == 1
     assert twq.launches_per_call("nope") == -1
 
 

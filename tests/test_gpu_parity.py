@@ -54,7 +54,30 @@ ADVERSARIAL = {
     "zero_groups": lambda: np.zeros((5, 512), np.float32),
     "all_equal": lambda: np.full((4, 256), -0.375, np.float32),
     "subnormal": lambda: np.tile((np.arange(128) + 1) * np.float32(2.0 ** -133), (2, 2)),
+    # scales above 2^125 (reciprocal not normal) and just inside the normal range
+    "huge": lambda: np.tile(np.linspace(-1.5, 1.5, 128, dtype=np.float32) * np.float32(2.0 ** 126), (2, 2)),
+    "tiny_normal": lambda: np.tile(np.linspace(-1.0, 1.0, 128, dtype=np.float32) * np.float32(2.0 ** -120), (2, 2)),
+    "tie_sweep": lambda: tie_sweep(72, 2048),
 }
+
+
+def tie_sweep(rows, m):
+    """Groups of 128 whose absmax a runs over all 128 BF16 mantissas of [1, 2) and
+    whose other elements run over every BF16 value of [a/16, a] of both signs, so
+    that v / s falls on or next to every half-integer the codes can round at."""
+    groups = rows * m // 128
+    out = np.empty((groups, 128), np.float32)
+    for gidx in range(groups):
+        k, chunk = gidx % 128, gidx // 128
+        a = np.float32(1.0 + k / 128.0)
+        mags = np.array([np.float32((1.0 + j / 128.0) * 2.0 ** e) for e in range(-4, 1)
+                         for j in range(128)], np.float32)
+        mags = mags[(mags <= a) & (mags >= a / 16)]
+        cand = np.concatenate([mags, -mags])
+        idx = (np.arange(127) + chunk * 127) % cand.size
+        out[gidx, 0] = a if chunk % 2 == 0 else -a
+        out[gidx, 1:] = cand[idx]
+    return out.reshape(rows, m)
 
 
 def _absmax_lanes():
@@ -94,6 +117,20 @@ def test_quantize_act_bitexact(twq, device, name, b):
     rq, rs = oracle.quantize_act(x)
     assert np.array_equal(xq.cpu().numpy(), rq)
     assert np.array_equal(sx.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    _status_clean(twq)
+
+
+def test_pack_weights_tie_sweep(twq, device):
+    # the same near-tie groups along the columns of R and L1 (offline packing path)
+    R = _bf16_exact(tie_sweep(128, 2048).T.copy())       # m = 2048, n = 128
+    L1 = _bf16_exact(tie_sweep(16, 2048).T.copy())       # m = 2048, r = 16
+    L2 = _bf16_exact(np.ones((16, 128), np.float32))
+    w = _pack(twq, device, R, L1, L2)
+    ref = oracle.pack_weights(R, L1, L2)
+    assert np.array_equal(w.rq.cpu().numpy(), ref["rq"])
+    assert np.array_equal(w.sr.cpu().numpy().view(np.uint32), ref["sr"].view(np.uint32))
+    assert np.array_equal(w.l1q.cpu().numpy(), ref["l1q"])
+    assert np.array_equal(w.sl1.cpu().numpy().view(np.uint32), ref["sl1"].view(np.uint32))
     _status_clean(twq)
 
 

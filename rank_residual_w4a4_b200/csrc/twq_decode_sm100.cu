@@ -96,12 +96,11 @@ static_assert(DLayout::kAlloc <= 227 * 1024, "shared memory budget");
 __device__ __forceinline__ void d_fail(int site) { atomicCAS(&g_decode_status, 0, site); }
 
 template <bool kCluster>
-__device__ __noinline__ bool d_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                    int site) {
+__device__ __noinline__ bool d_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         int site) {
   auto probe = [&]() {
     return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
   };
-  if (probe()) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
@@ -114,6 +113,16 @@ __device__ __noinline__ bool d_wait(uint64_t* bar, uint32_t parity, volatile int
       return false;
     }
   }
+}
+
+// Bounded wait for `parity` on `bar`: one inline probe (the common case on the
+// issuing threads, where the phase has often completed already), then the
+// bounded loop. Gives up after kWaitLimitNs or once the CTA's abort flag is set.
+template <bool kCluster>
+__device__ __forceinline__ bool d_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                       int site) {
+  if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  return d_wait_slow<kCluster>(bar, parity, abort_flag, site);
 }
 
 __device__ __forceinline__ uint8_t* d_align1024(uint8_t* p) {
@@ -149,51 +158,67 @@ __device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int j, uin
 
 // Eq. (1) quantizer fused into the prologue. The CTA's BF16 slice of X sits in
 // shared memory as two TMA boxes per group (64 elements x 16 tokens each, rows
-// of 128 bytes; tokens >= b read as zero). Half-warp `hw` of the 20 turns the
-// (token, group) pairs hw, hw + 20, ... into int8 codes (16*q, in the in-chunk
-// order of unpack8) in the 128-byte-swizzle B tiles and fp32 scales in sxs,
-// with the arithmetic of twq_quantize_act, so the codes are identical.
-constexpr int kQHalfWarps = 20;  // quantizing half-warps: warps 2-3 and 12-19
+// of 128 bytes; tokens >= b read as zero). Eight lanes take one (token, group)
+// pair, 16 elements each; quantizing lane `qi` of 80 (warps 2-3 and 12-19)
+// handles the pairs qi / 8 + 10 k. Codes go to the 128-byte-swizzle B tiles as
+// 16*q in the in-chunk order of unpack8, scales to sxs, with the arithmetic of
+// twq_quantize_act, so the codes are identical.
+constexpr int kQPairsPerPass = 40;  // 10 warps x 4 pairs
 
 __device__ __forceinline__ void quantize_slice(const uint8_t* xs, int ng, uint8_t* xu, float* sxs,
-                                               int hw, int lane) {
-  const int l = lane & 15;
+                                               uint64_t* xready, int qi, int lane) {
+  const int l = lane & 7;  // elements [16 l, 16 l + 16) of the group
   const int pairs = kNT * ng;
-  const int iters = (pairs + kQHalfWarps - 1) / kQHalfWarps;  // the same for both halves of a warp
+  const int passes = (pairs + kQPairsPerPass - 1) / kQPairsPerPass;  // uniform over the warp
 #pragma unroll 1
-  for (int it = 0; it < iters; ++it) {
-    const int p = hw + it * kQHalfWarps;
+  for (int it = 0; it < passes; ++it) {
+    const int p = (qi >> 3) + it * kQPairsPerPass;
     const bool pv = p < pairs;
     const int gi = pv ? p / kNT : 0, t = pv ? p % kNT : 0;
-    const uint4 raw = *reinterpret_cast<const uint4*>(xs + gi * 4096 + (l >> 3) * 2048 + t * 128 +
-                                                      (l & 7) * 16);
-    float f[8];
-    f[0] = __uint_as_float(raw.x << 16);
-    f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-    f[2] = __uint_as_float(raw.y << 16);
-    f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-    f[4] = __uint_as_float(raw.z << 16);
-    f[5] = __uint_as_float(raw.z & 0xFFFF0000u);
-    f[6] = __uint_as_float(raw.w << 16);
-    f[7] = __uint_as_float(raw.w & 0xFFFF0000u);
-    float a = 0.0f;
+    const uint8_t* src = xs + gi * 4096 + (l >> 2) * 2048 + t * 128 + (l & 3) * 32;
+    const uint4 r0 = *reinterpret_cast<const uint4*>(src);
+    const uint4 r1 = *reinterpret_cast<const uint4*>(src + 16);
+    const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    // f[0..7]: even elements 0, 2, .., 14 of the lane's 16; f[8..15]: odd elements
+    float f[16];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(f[k]));
+    for (int i = 0; i < 8; ++i) {
+      f[i] = __uint_as_float(w[i] << 16);
+      f[8 + i] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+    float m4[4];  // absmax as a tree, for instruction-level parallelism
 #pragma unroll
-    for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+    for (int i = 0; i < 4; ++i)
+      m4[i] = fmaxf(fmaxf(fabsf(f[i]), fabsf(f[i + 4])), fmaxf(fabsf(f[i + 8]), fabsf(f[i + 12])));
+    float a = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
     const Eq1Scale ks = eq1_scale(a);
-    uint32_t w0 = 0, w1 = 0;
+    uint4 o = make_uint4(0, 0, 0, 0);
     if (ks.s != 0.0f) {
-      float c[8];
-      eq1_codes8(f, ks, c);
-      w0 = (eq1_nibble(c[0]) << 4) | (eq1_nibble(c[2]) << 12) | (eq1_nibble(c[4]) << 20) |
-           (eq1_nibble(c[6]) << 28);
-      w1 = (eq1_nibble(c[1]) << 4) | (eq1_nibble(c[3]) << 12) | (eq1_nibble(c[5]) << 20) |
-           (eq1_nibble(c[7]) << 28);
+      uint32_t nb[16];
+      eq1_nibbles(f, ks, nb);
+      // 16*q bytes: even elements 0..6, odd 1..7, even 8..14, odd 9..15
+      o.x = (nb[0] << 4) | (nb[1] << 12) | (nb[2] << 20) | (nb[3] << 28);
+      o.y = (nb[8] << 4) | (nb[9] << 12) | (nb[10] << 20) | (nb[11] << 28);
+      o.z = (nb[4] << 4) | (nb[5] << 12) | (nb[6] << 20) | (nb[7] << 28);
+      o.w = (nb[12] << 4) | (nb[13] << 12) | (nb[14] << 20) | (nb[15] << 28);
     }
     if (pv) {
-      *reinterpret_cast<uint2*>(xu + gi * 2048 + d_sw128(t, l >> 1) + (l & 1) * 8) = make_uint2(w0, w1);
+      *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(t, l)) = o;
       if (l == 0) sxs[gi * kNT + t] = ks.s;
+    }
+    // Groups whose last pair falls in this pass are complete once every warp
+    // has passed here: each warp arrives once on each of them.
+    const int g_lo = it * kQPairsPerPass / kNT;
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      for (int g = g_lo; g < ng; ++g) {
+        const int done_pass = (g * kNT + kNT - 1) / kQPairsPerPass;
+        if (done_pass == it) mbar_arrive(&xready[g]);
+        if (done_pass > it) break;
+      }
     }
   }
 }
@@ -234,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* h_full = ar_empty + kRing;        // [kMaxGroups] stage-1 accumulator ready
   uint64_t* res_full = h_full + kMaxGroups;   // [kMaxGroups] residual accumulator ready
   uint64_t* xfull = res_full + kMaxGroups;
-  uint64_t* xready = xfull + 1;
-  uint64_t* l2full = xready + 1;
+  uint64_t* xready = xfull + 1;               // [kMaxGroups] group's X codes and scales ready
+  uint64_t* l2full = xready + kMaxGroups;
   uint64_t* hb_ready = l2full + 1;
   uint64_t* lr_full = hb_ready + 1;
   uint64_t* h_ready = lr_full + 1;
@@ -267,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // barrier init spread over the warp: lane i owns group i's copy barriers
     if (lane < kMaxGroups) {
+      mbar_init(&xready[lane], kQ ? 10 : 2);
       mbar_init(&rfull[lane], 1);
       mbar_init(&lfull[lane], 1);
       mbar_init(&h_full[lane], 1);
@@ -280,7 +306,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 31) {
       mbar_init(xfull, 1);
-      mbar_init(xready, kQ ? 10 : 2);
       mbar_init(l2full, 1);
       mbar_init(hb_ready, 4);
       mbar_init(lr_full, 1);
@@ -345,18 +370,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (kQ && (warp == 2 || warp == 3 || warp >= 12)) {
     // ----- X quantize (warps 2-3 and 12-19; 12-19 then go on to their own roles)
-    const int hw = (warp < 4 ? warp - 2 : warp - 10) * 2 + (lane >> 4);
-    if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) {
-      quantize_slice(xp, ng, xu, sxs, hw, lane);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xready);
-    }
+    const int qi = (warp < 4 ? warp - 2 : warp - 10) * 32 + lane;
+    if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) quantize_slice(xp, ng, xu, sxs, xready, qi, lane);
   }
   if (warp == 0) {
     // ------------------------------------ residual MMA issuer (lane 0 of warp 0)
     if (lane == 0) {
-      bool ok = d_wait<false>(xready, 0, abort_flag, kDSiteX);
+      bool ok = true;
       const uint32_t xu0 = smem_u32(xu);
       const uint32_t idesc = idesc_i8(kNT);
       if (T::res) {
@@ -364,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int slot = gi % kRing;
           const uint32_t ph = (gi / kRing) & 1;
           const uint64_t db = smem_desc_sw128(xu0 + gi * 2048);
+          if (!(ok = d_wait<false>(&xready[gi], 0, abort_flag, kDSiteX))) break;
           if (!(ok = d_wait<false>(&ar_full[slot], ph, abort_flag, kDSiteAr))) break;
           tc_fence_after();
 #pragma unroll
@@ -388,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool ok = d_wait<false>(xready, 0, abort_flag, kDSiteX);
+      bool ok = true;
       const uint32_t xu0 = smem_u32(xu);
       const uint32_t idesc = idesc_i8(kNT);
       for (int gi = 0; gi < ng && ok; ++gi) {
@@ -396,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (gi / kRing) & 1;
         const uint64_t db = smem_desc_sw128(xu0 + gi * 2048);
         if (T::lr) {
+          if (!(ok = d_wait<false>(&xready[gi], 0, abort_flag, kDSiteX))) break;
           if (!(ok = d_wait<false>(&al_full[slot], ph, abort_flag, kDSiteAl))) break;
           tc_fence_after();
 #pragma unroll
@@ -449,7 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) sxs[tid + 64 * i] = sxv[i];
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(xready);
+        if (lane == 0)
+          for (int g = 0; g < ng; ++g) mbar_arrive(&xready[g]);
       }
     }
   } else if (warp < 12) {
@@ -491,7 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float acc[kNT];
 #pragma unroll
       for (int t = 0; t < kNT; ++t) acc[t] = 0.0f;
-      bool ok = d_wait<false>(xready, 0, abort_flag, kDSiteX);
+      // every quantizing warp arrives on the last group's barrier after all its scale
+      // writes, so one wait makes every group's sxs visible
+      bool ok = ng == 0 || d_wait<false>(&xready[ng - 1], 0, abort_flag, kDSiteX);
 #pragma unroll
       for (int gi = 0; gi < kMaxGroups; ++gi) {
         if (gi < ng && ok) {
@@ -555,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float acc[kNT];
 #pragma unroll
     for (int t = 0; t < kNT; ++t) acc[t] = 0.0f;
-    bool ok = d_wait<false>(xready, 0, abort_flag, kDSiteX);
+    bool ok = !T::res || ng == 0 || d_wait<false>(&xready[ng - 1], 0, abort_flag, kDSiteX);
     if (T::res) {
       float srv[kMaxGroups];
 #pragma unroll

@@ -52,10 +52,10 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
   const float s = ks.s;
   uint32_t word = 0;
   if (s != 0.0f) {
-    float t[8];
-    eq1_codes8(f, ks, t);
+    uint32_t nib[8];
+    eq1_nibbles(f, ks, nib);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) word |= eq1_nibble(t[k]) << (4 * k);
+    for (int k = 0; k < 8; ++k) word |= nib[k] << (4 * k);
   }
   if (valid) {
     *reinterpret_cast<uint32_t*>(xq + row * (m / 2) + g * 64 + l * 4) = word;
@@ -85,13 +85,14 @@ __global__ void __launch_bounds__(128) pack_cols_kernel(const uint16_t* __restri
     for (int wi = 0; wi < 4; ++wi) {
       uint32_t word = 0;
       if (sc != 0.0f) {
-        float v[8], t[8];
+        float v[8];
+        uint32_t nib[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           v[k] = bf16_bits_to_f32(__ldg(p + static_cast<int64_t>(c * 32 + wi * 8 + k) * cols));
-        eq1_codes8(v, ks, t);
+        eq1_nibbles(v, ks, nib);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) word |= eq1_nibble(t[k]) << (4 * k);
+        for (int k = 0; k < 8; ++k) word |= nib[k] << (4 * k);
       }
       words[wi] = word;
     }

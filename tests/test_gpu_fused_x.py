@@ -11,7 +11,7 @@ import pytest
 import oracle
 import synth
 from helpers import assert_y_close, bits_of, to_dev
-from test_gpu_parity import tie_sweep
+from test_gpu_parity import every_absmax, tie_sweep
 
 pytestmark = pytest.mark.gpu
 
@@ -117,6 +117,19 @@ def test_fused_x_adversarial_inputs(twq, device, case):
     xd = to_dev(x, device)
     y = bits_of(twq.fused_linear_x(xd, w))
     assert np.array_equal(y, _two_call(twq, xd, w)), case
+    _status_clean(twq)
+
+
+def test_fused_x_every_absmax(twq, device):
+    # every BF16 absmax through the in-kernel quantizer: 16 tokens x 64 groups per call
+    b, m, n, r = 16, 8192, 128, 16
+    _, R, L1, L2 = _operands(b, m, n, r, seed=26)
+    w = _pack(twq, device, R, L1, L2)
+    allx = synth.f32_to_bf16(every_absmax(16 * 32, m))
+    for c in range(32):
+        xd = to_dev(allx[16 * c:16 * c + 16], device)
+        y = bits_of(twq.fused_linear_x(xd, w))
+        assert np.array_equal(y, _two_call(twq, xd, w)), "chunk %d" % c
     _status_clean(twq)
 
 

@@ -58,6 +58,7 @@ ADVERSARIAL = {
     "huge": lambda: np.tile(np.linspace(-1.5, 1.5, 128, dtype=np.float32) * np.float32(2.0 ** 126), (2, 2)),
     "tiny_normal": lambda: np.tile(np.linspace(-1.0, 1.0, 128, dtype=np.float32) * np.float32(2.0 ** -120), (2, 2)),
     "tie_sweep": lambda: tie_sweep(72, 2048),
+    "every_absmax": lambda: every_absmax(256, 16384),
 }
 
 
@@ -78,6 +79,22 @@ def tie_sweep(rows, m):
         out[gidx, 0] = a if chunk % 2 == 0 else -a
         out[gidx, 1:] = cand[idx]
     return out.reshape(rows, m)
+
+
+def every_absmax(rows, m, seed=9):
+    """Groups whose absmax runs over every non-negative finite BF16 value (32,640 of
+    them, zero included), at a lane that moves from group to group, with the other
+    elements below it; the leftover groups are zero."""
+    groups = rows * m // 128
+    assert groups >= 0x7F80
+    rng = np.random.default_rng(seed)
+    a = np.zeros(groups, np.float32)
+    a[:0x7F80] = (np.arange(0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    f = (a[:, None] * rng.uniform(-1, 1, (groups, 128))).astype(np.float32)
+    pos = (np.arange(groups) * 37) % 128
+    sign = np.where(np.arange(groups) % 2 == 0, 1.0, -1.0).astype(np.float32)
+    f[np.arange(groups), pos] = sign * a
+    return f.reshape(rows, m)
 
 
 def _absmax_lanes():
@@ -117,6 +134,17 @@ def test_quantize_act_bitexact(twq, device, name, b):
     rq, rs = oracle.quantize_act(x)
     assert np.array_equal(xq.cpu().numpy(), rq)
     assert np.array_equal(sx.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    _status_clean(twq)
+
+
+def test_pack_weights_every_absmax(twq, device):
+    # every BF16 absmax as a (group, column) scale of R: m = 2048, n = 2048
+    R = _bf16_exact(every_absmax(2048, 2048).reshape(2048, 16, 128).transpose(1, 2, 0)
+                    .reshape(2048, 2048).copy())
+    w = _pack(twq, device, R, None, None)
+    ref = oracle.pack_weights(R, None, None)
+    assert np.array_equal(w.rq.cpu().numpy(), ref["rq"])
+    assert np.array_equal(w.sr.cpu().numpy().view(np.uint32), ref["sr"].view(np.uint32))
     _status_clean(twq)
 
 

@@ -95,21 +95,32 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    # the files a capture of each kernel depends on
+    "decode": ("twq_decode_sm100.cu", "sm100_ptx.cuh", "twq_eq1.cuh"),
+    "gemm": ("twq_gemm_sm100.cu", "sm100_ptx.cuh"),
+}
+
+
+def kernel_source_hash(kind):
     h = hashlib.sha256()
-    for f in ("twq_gemm_sm100.cu", "twq_decode_sm100.cu", "sm100_ptx.cuh"):
+    for f in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, "rank_residual_w4a4_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
+def kernel_kind(workload):
+    return "decode" if describe(workload.replace("_x", ""))[1] <= 16 else "gemm"
+
+
 def profiled_traffic(workload):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary, or None
-    if the summary has no line for this workload or the kernel source changed since."""
+    """DRAM bytes per launch of the layer kernel from the committed ncu summary, or None
+    if the summary has no line for this workload or the kernel's sources changed since."""
     p = os.path.join(ROOT, "profiles", "fused_kernel_traffic.txt")
     if not os.path.exists(p):
         return None
-    want = kernel_source_hash()
+    want = kernel_source_hash(kernel_kind(workload))
     with open(p) as fh:
         for line in fh:
             parts = line.split()

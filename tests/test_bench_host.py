@@ -34,12 +34,13 @@ def test_roofline_entries():
 
 
 def test_traffic_table_is_tied_to_the_kernel_sources():
-    h = bench.kernel_source_hash()
     path = os.path.join(bench.ROOT, "profiles", "fused_kernel_traffic.txt")
     lines = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
     for wl, nbytes, hh in lines:
+        h = bench.kernel_source_hash(bench.kernel_kind(wl))
         got = bench.profiled_traffic(wl)
         assert got == (int(nbytes) if hh == h else None)
+    assert bench.kernel_kind("decode16_x") == "decode" and bench.kernel_kind("gateup") == "gemm"
 
 
 def _rank_main(rank, world, port, out):

@@ -126,6 +126,15 @@ __device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile i
   }
 }
 
+// wait_bar with the first probe inline, for the single-thread producer and MMA
+// roles, where the phase has often completed already and a call costs more than
+// the probe.
+__device__ __forceinline__ bool wait_fast(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bar(bar, parity, abort_flag, site);
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -136,37 +145,54 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int c) {
 }
 
 // 4-bit codes (rows x 64 bytes, dense) -> int8 (rows x 128 bytes, swizzled), 16*q per byte.
-// Each thread takes 16 packed bytes (two 16-byte output chunks) per item, and
-// four items are loaded before any is stored so the shared-memory latencies
-// overlap.
-__device__ __forceinline__ void unpack_rows(const uint8_t* src, uint8_t* dst, int rows, int tid,
-                                            int nthreads) {
-  const int items = rows * 4;  // 16 packed bytes each
-  for (int e0 = tid; e0 < items; e0 += 4 * nthreads) {
-    uint4 w[4];
+// A thread of the 192 unpack threads takes the 16-byte items tid, tid + 192 and
+// tid + 384 of a 128-row tile (an item: 16 packed bytes of one row, two output
+// chunks). The offsets depend only on the thread, so they are computed once.
+constexpr int kUnpackThreads = 192;
+struct UnpackPlan {
+  uint32_t src[3];     // byte offset of the item in the packed tile
+  uint32_t dst0[3];    // swizzled offsets of its two output chunks
+  uint32_t dst1[3];
+  int row[3];          // tile row of the item (>= 128: no item)
+};
+
+__device__ __forceinline__ UnpackPlan unpack_plan(int tid) {
+  UnpackPlan p;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = e0 + i * nthreads;
-      if (e < items) w[i] = *reinterpret_cast<const uint4*>(src + e * 16);
-    }
+  for (int i = 0; i < 3; ++i) {
+    const int e = tid + i * kUnpackThreads;
+    const int row = e >> 2;
+    const int c = (e & 3) * 2;
+    p.row[i] = row;
+    p.src[i] = static_cast<uint32_t>(e * 16);
+    p.dst0[i] = sw128_offset(row & 127, c);
+    p.dst1[i] = sw128_offset(row & 127, c + 1);
+  }
+  return p;
+}
+
+// Unpacks the first `rows` rows (<= 128) of a tile with the thread's plan; all
+// loads are issued before any store so the shared-memory latencies overlap.
+__device__ __forceinline__ void unpack_tile(const uint8_t* src, uint8_t* dst, int rows,
+                                            const UnpackPlan& p) {
+  uint4 w[3];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = e0 + i * nthreads;
-      if (e < items) {
-        const int row = e >> 2;
-        const int c = (e & 3) * 2;
-        uint4 o0, o1;
-        o0.x = (w[i].x << 4) & 0xF0F0F0F0u;
-        o0.y = w[i].x & 0xF0F0F0F0u;
-        o0.z = (w[i].y << 4) & 0xF0F0F0F0u;
-        o0.w = w[i].y & 0xF0F0F0F0u;
-        o1.x = (w[i].z << 4) & 0xF0F0F0F0u;
-        o1.y = w[i].z & 0xF0F0F0F0u;
-        o1.z = (w[i].w << 4) & 0xF0F0F0F0u;
-        o1.w = w[i].w & 0xF0F0F0F0u;
-        *reinterpret_cast<uint4*>(dst + sw128_offset(row, c)) = o0;
-        *reinterpret_cast<uint4*>(dst + sw128_offset(row, c + 1)) = o1;
-      }
+  for (int i = 0; i < 3; ++i)
+    if (p.row[i] < rows) w[i] = *reinterpret_cast<const uint4*>(src + p.src[i]);
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    if (p.row[i] < rows) {
+      uint4 o0, o1;
+      o0.x = (w[i].x << 4) & 0xF0F0F0F0u;
+      o0.y = w[i].x & 0xF0F0F0F0u;
+      o0.z = (w[i].y << 4) & 0xF0F0F0F0u;
+      o0.w = w[i].y & 0xF0F0F0F0u;
+      o1.x = (w[i].z << 4) & 0xF0F0F0F0u;
+      o1.y = w[i].z & 0xF0F0F0F0u;
+      o1.z = (w[i].w << 4) & 0xF0F0F0F0u;
+      o1.w = w[i].w & 0xF0F0F0F0u;
+      *reinterpret_cast<uint4*>(dst + p.dst0[i]) = o0;
+      *reinterpret_cast<uint4*>(dst + p.dst1[i]) = o1;
     }
   }
 }
@@ -335,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int hc = 0; hc < HC && ok; ++hc) {
             const int nh = min(kHChunk, args.r - hc * kHChunk);
             for (int g = 0; g < G; ++g) {
-              if (!(ok = wait_bar(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
+              if (!(ok = wait_fast(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
                 break;
               uint8_t* slot = slots + s.idx * L::kSlot;
               mbar_arrive_expect_tx(&full[s.idx], L::kSlotA + args.h_box * 64);
@@ -344,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               pend[s.idx] = true;
               pend_phase[s.idx] = s.phase;
               s.next(kPackedStages);
-              if (!(ok = wait_bar(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
+              if (!(ok = wait_fast(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
                                   kSiteProducerScaleEmpty)))
                 break;
               mbar_arrive_expect_tx(&sc_full[q.idx], nh * 4);
@@ -358,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (T::res && ok) {
           for (int g = 0; g < G; ++g) {
-            if (!(ok = wait_bar(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
+            if (!(ok = wait_fast(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
               break;
             uint8_t* slot = slots + s.idx * L::kSlot;
             mbar_arrive_expect_tx(&full[s.idx], L::kSlotA + BN * 64);
@@ -367,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pend[s.idx] = true;
             pend_phase[s.idx] = s.phase;
             s.next(kPackedStages);
-            if (!(ok = wait_bar(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
+            if (!(ok = wait_fast(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
                                 kSiteProducerScaleEmpty)))
               break;
             mbar_arrive_expect_tx(&sc_full[q.idx], BN * 4);
@@ -380,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (T::s2 && ok) {
           if (T::h_global) {
-            if (!(ok = wait_bar(hb_free, hb_phase ^ 1u, abort_flag, kSiteProducerHbFree))) break;
+            if (!(ok = wait_fast(hb_free, hb_phase ^ 1u, abort_flag, kSiteProducerHbFree))) break;
             mbar_arrive_expect_tx(hb_ready, KC * 16384);
             for (int kc = 0; kc < KC; ++kc)
               tma_load_2d(hb + kc * 16384, &tm_h, hb_ready, kc * 64, row0);
@@ -388,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             hb_phase ^= 1u;
           }
           for (int kc = 0; kc < KC; ++kc) {
-            if (!(ok = wait_bar(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
+            if (!(ok = wait_fast(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
               break;
             mbar_arrive_expect_tx(&full[s.idx], BN * 128);
             tma_load_2d(slots + s.idx * L::kSlot, &tm_l2t, &full[s.idx], kc * 64, n0);
@@ -403,10 +429,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int dummy = 0;
         volatile int* never = &dummy;
         for (int i = 0; i < kPackedStages; ++i)
-          if (pend[i]) wait_bar(&full[i], pend_phase[i], never, kSiteFinal);
+          if (pend[i]) wait_fast(&full[i], pend_phase[i], never, kSiteFinal);
         for (int i = 0; i < kScaleSlots; ++i)
-          if (spend[i]) wait_bar(&sc_full[i], spend_phase[i], never, kSiteFinal);
-        if (T::h_global && hb_pend) wait_bar(hb_ready, hb_phase ^ 1u, never, kSiteFinal);
+          if (spend[i]) wait_fast(&sc_full[i], spend_phase[i], never, kSiteFinal);
+        if (T::h_global && hb_pend) wait_fast(hb_ready, hb_phase ^ 1u, never, kSiteFinal);
       }
     }
   } else if (warp == 1) {
@@ -424,8 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nh = min(kHChunk, args.r - hc * kHChunk);
             const uint32_t idesc = idesc_i8(nh);
             for (int g = 0; g < G; ++g) {
-              if (!(ok = wait_bar(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
-              if (!(ok = wait_bar(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
+              if (!(ok = wait_fast(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
+              if (!(ok = wait_fast(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
                 break;
               tc_fence_after();
               const uint32_t d = tmem_base + a.idx * BN;
@@ -443,8 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (T::res && ok) {
           const uint32_t idesc = idesc_i8(BN);
           for (int g = 0; g < G; ++g) {
-            if (!(ok = wait_bar(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
-            if (!(ok = wait_bar(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
+            if (!(ok = wait_fast(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
+            if (!(ok = wait_fast(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
               break;
             tc_fence_after();
             const uint32_t d = tmem_base + a.idx * BN;
@@ -460,15 +486,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (T::s2 && ok) {
           if (ti.need_h || T::h_global) {
-            if (!(ok = wait_bar(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) break;
+            if (!(ok = wait_fast(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) break;
             hb_phase ^= 1u;
           }
-          if (!(ok = wait_bar(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
+          if (!(ok = wait_fast(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
             break;
           const uint32_t idesc = idesc_bf16(BN);
           const uint32_t d = tmem_base + a.idx * BN;
           for (int kc = 0; kc < KC; ++kc) {
-            if (!(ok = wait_bar(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
+            if (!(ok = wait_fast(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
             tc_fence_after();
             const uint64_t da = smem_desc_sw128(hb0 + kc * 16384);
             const uint64_t db = smem_desc_sw128(ua0 + u.idx * L::kUStage + L::kUA);
@@ -487,11 +513,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // All MMAs issued by this thread are complete before TMEM is released.
       mma_commit(mma_done);
       int dummy = 0;
-      wait_bar(mma_done, 0, &dummy, kSiteFinal);
+      wait_fast(mma_done, 0, &dummy, kSiteFinal);
     }
   } else if (warp >= 2 && warp < 8) {
     // --------------------------------------------------------------- unpack
+    static_assert(kBM == 128 && BN == 128, "the unpack plan covers 128-row tiles");
     const int tid = threadIdx.x - 64;
+    const UnpackPlan plan = unpack_plan(tid);
     Ring s, u;
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t) {
@@ -510,8 +538,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int hc = step / G;
             brows = min(kHChunk, args.r - hc * kHChunk);
           }
-          unpack_rows(src, dst, kBM, tid, 192);
-          unpack_rows(src + L::kSlotA, dst + L::kUA, brows, tid, 192);
+          unpack_tile(src, dst, kBM, plan);
+          unpack_tile(src + L::kSlotA, dst + L::kUA, brows, plan);
         } else {
           copy_smem(src, dst + L::kUA, BN * 128, tid, 192);
         }

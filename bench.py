@@ -539,10 +539,47 @@ def sweep(args, device, peaks):
         out.append(res)
         del prob, ws
         torch.cuda.empty_cache()
+    out.append(fold_entry(device))
     st = twq.device_status()
     if st != 0:
         raise RuntimeError("device wait timed out at site %d" % st)
     return out
+
+
+# fp32 CUDA-core peak of the fold's GEMMs: 148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def fold_entry(device, m=4096, n=4096, r=128, reps=3):
+    """The offline transform fold (U' = Q^T U G, V' = G^-1 V, R' = Q^T R) at the
+    decode layer's dimensions: plain fp32 CUDA-core GEMMs, bound by fp32 issue."""
+    import torch
+    from rank_residual_w4a4_b200 import twq
+    g = torch.Generator(device="cpu").manual_seed(0)
+    Q = torch.linalg.qr(torch.randn(m, m, generator=g, dtype=torch.float64))[0].float().contiguous().to(device)
+    G = (torch.eye(r, dtype=torch.float64) + 0.25 * torch.randn(r, r, generator=g, dtype=torch.float64)
+         / r ** 0.5).float().to(device)
+    U = (0.05 * torch.randn(m, r, generator=g)).to(torch.bfloat16).to(device)
+    V = (0.05 * torch.randn(r, n, generator=g)).to(torch.bfloat16).to(device)
+    R = (0.02 * torch.randn(m, n, generator=g)).to(torch.bfloat16).to(device)
+    ws = torch.empty(twq.fold_workspace_bytes(m, n, r), dtype=torch.uint8, device=device)
+    twq.fold_transforms(Q, G, U, V, R, ws)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        twq.fold_transforms(Q, G, U, V, R, ws)
+    e.record()
+    torch.cuda.synchronize()
+    t = s.elapsed_time(e) / 1e3 / reps
+    flops = 2.0 * (m * r * r + m * m * r + r * r * n + m * m * n)
+    ach = flops / t / 1e12
+    return {"workload": "fold m=%d n=%d r=%d" % (m, n, r), "fold_ms": round(t * 1e3, 3),
+            "roofline": {"bound": "alu", "achieved": round(ach, 2), "peak": round(FP32_ALU_PEAK_TFLOPS, 1),
+                         "unit": "TFLOP/s", "frac": round(ach / FP32_ALU_PEAK_TFLOPS, 4),
+                         "traffic": None,
+                         "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz"},
+            "timing": "events around %d calls (each synchronizes once)" % reps}
 
 
 # ------------------------------------------------------------- CPU oracle arm

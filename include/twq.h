@@ -22,7 +22,8 @@
  *            merges both components).
  *
  * Memory: every pointer is a DEVICE pointer owned by the caller; the library
- * never allocates, frees or synchronizes (except twq_device_status). Every
+ * never allocates, frees or synchronizes (except twq_device_status and the
+ * offline twq_fold_transforms). Every
  * call is asynchronous on `stream`; inputs must stay live until the stream
  * reaches the call. All base pointers must be 16-byte aligned.
  *
@@ -202,6 +203,30 @@ TWQ_API twq_status twq_unfused_linear(const uint8_t* xq, const float* sx, int64_
 TWQ_API twq_status twq_unfused_linear_noalloc(const uint8_t* xq, const float* sx, int64_t b,
                                               const twq_weights* w, uint16_t* y,
                                               twq_stream_t stream);
+
+/*
+ * Offline fold of the learned transforms into the layer's factors (TwinQuant
+ * §4.1, Eq. (6) and the factors after it: U' = Q^-1 U G, V' = G^-1 V,
+ * R' = Q^-1 R, absorbed offline). The layer then runs on X' = X Q with
+ * L1 = U', L2 = V', R = R' (twq_pack_weights). Not on the per-token path.
+ *   Q   m x m fp32 row-major, orthogonal (§4.2: Q^T Q = I), so Q^-1 = Q^T
+ *   G   r x r fp32 row-major, invertible; inverted on the device by Gauss-Jordan
+ *       elimination with partial pivoting in fp64
+ *   U   m x r, V r x n, R m x n: BF16 row-major (the decomposed factors)
+ *   L1_out m x r, L2_out r x n, R_out m x n: BF16 row-major outputs (RNE of
+ *       products accumulated in fp32)
+ *   workspace: device buffer of twq_fold_workspace_bytes(m, n, r) bytes,
+ *       256-byte aligned
+ * Limits: r <= 1024, m <= 4,194,240. This call SYNCHRONIZES `stream` (it reads
+ * back whether G was singular): TWQ_ERR_INVALID_ARG if a pivot column of G
+ * has no nonzero entry (the outputs are then unspecified).
+ */
+TWQ_API size_t twq_fold_workspace_bytes(int64_t m, int64_t n, int64_t r);
+TWQ_API twq_status twq_fold_transforms(const float* Q, const float* G, const uint16_t* U,
+                                       const uint16_t* V, const uint16_t* R, int64_t m, int64_t n,
+                                       int64_t r, uint16_t* L1_out, uint16_t* L2_out,
+                                       uint16_t* R_out, void* workspace, size_t workspace_bytes,
+                                       twq_stream_t stream);
 
 /*
  * Reads and clears the device-side status word (SYNCHRONIZES the device).

@@ -213,3 +213,32 @@ def layer(x_bits, R, L1, L2, mode=FUSED, rows=None, want=("y",)):
         ql1 = sl1 = None
         L2 = None
     return linear(qx, sx, qr, sr, ql1, sl1, L2, mode=mode, rows=rows, want=want)
+
+
+def _bf16_to_f64(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _f64_to_bf16(f):
+    """fp64 -> fp32 (RNE) -> BF16 (RNE) bit patterns, finite inputs."""
+    u = np.asarray(f, np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def fold_transforms(Q, G, U, V, R, rounded=True):
+    """Offline fold of TwinQuant §4.1 (Eq. (6) and the factors after it):
+    U' = Q^-1 U G, V' = G^-1 V, R' = Q^-1 R, with Q orthogonal (§4.2: Q^T Q = I,
+    read as Q^-1 = Q^T) and G invertible (G^-1 by numpy's LU inverse).
+
+    Q: m x m fp32, G: r x r fp32; U (m x r), V (r x n), R (m x n): BF16 bits.
+    Returns BF16 bits of (U', V', R') in fp64 arithmetic, or the fp64 values
+    themselves if not `rounded`."""
+    q = np.asarray(Q, np.float32).astype(np.float64)
+    g = np.asarray(G, np.float32).astype(np.float64)
+    u, v, r = _bf16_to_f64(U), _bf16_to_f64(V), _bf16_to_f64(R)
+    l1 = q.T @ (u @ g)
+    l2 = np.linalg.inv(g) @ v
+    rr = q.T @ r
+    if not rounded:
+        return l1, l2, rr
+    return _f64_to_bf16(l1), _f64_to_bf16(l2), _f64_to_bf16(rr)

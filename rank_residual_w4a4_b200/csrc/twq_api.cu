@@ -218,6 +218,7 @@ int twq_launches_per_call(const char* ep) {
       !strcmp(ep, "twq_lowrank_only") || !strcmp(ep, "twq_fused_linear_x"))
     return 1;
   if (!strcmp(ep, "twq_unfused_linear") || !strcmp(ep, "twq_unfused_linear_noalloc")) return 4;
+  if (!strcmp(ep, "twq_fold_transforms")) return 5;
   return -1;
 }
 

@@ -27,7 +27,7 @@ EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_siz
            "twq_quantize_act", "twq_pack_weights", "twq_fused_linear", "twq_w4a4_only",
            "twq_lowrank_only", "twq_unfused_workspace_bytes", "twq_unfused_linear",
            "twq_device_status", "twq_launches_per_call", "twq_unfused_linear_noalloc",
-           "twq_fused_linear_x")
+           "twq_fused_linear_x", "twq_fold_workspace_bytes", "twq_fold_transforms")
 
 
 class TwqError(RuntimeError):
@@ -71,6 +71,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twq_launches_per_call": ([ctypes.c_char_p], ctypes.c_int),
         "twq_unfused_linear_noalloc": ([P, P, I, P, P, P], ctypes.c_int),
         "twq_fused_linear_x": ([P, I, I, P, P, P], ctypes.c_int),
+        "twq_fold_workspace_bytes": ([I, I, I], S),
+        "twq_fold_transforms": ([P, P, P, P, P, I, I, I, P, P, P, P, S, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -208,6 +210,30 @@ def fused_linear_x(x: torch.Tensor, w: Weights, y=None, stream=None):
                                      _dev(y, "y", torch.bfloat16), _stream(stream)),
            "twq_fused_linear_x")
     return y
+
+
+def fold_workspace_bytes(m: int, n: int, r: int) -> int:
+    return int(load().twq_fold_workspace_bytes(m, n, r))
+
+
+def fold_transforms(Q, G, U, V, R, workspace=None, stream=None):
+    """Offline fold U' = Q^T U G, V' = G^-1 V, R' = Q^T R (BF16 outputs); synchronizes."""
+    m, r = U.shape
+    n = V.shape[1]
+    dev = U.device
+    out = (torch.empty((m, r), dtype=torch.bfloat16, device=dev),
+           torch.empty((r, n), dtype=torch.bfloat16, device=dev),
+           torch.empty((m, n), dtype=torch.bfloat16, device=dev))
+    nbytes = fold_workspace_bytes(m, n, r)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(load().twq_fold_transforms(
+        _dev(Q, "Q", torch.float32), _dev(G, "G", torch.float32), _dev(U, "U", torch.bfloat16),
+        _dev(V, "V", torch.bfloat16), _dev(R, "R", torch.bfloat16), m, n, r,
+        _dev(out[0], "L1_out", torch.bfloat16), _dev(out[1], "L2_out", torch.bfloat16),
+        _dev(out[2], "R_out", torch.bfloat16), _dev(workspace, "workspace", torch.uint8),
+        workspace.numel(), _stream(stream)), "twq_fold_transforms")
+    return out
 
 
 def w4a4_only(xq, sx, w: Weights, y=None, stream=None):

@@ -125,6 +125,21 @@ def test_fused_linear_x_validation(lib):
     assert f(A, 512, 4, ctypes.byref(big), A, None) == 2
 
 
+def test_fold_validation(lib):
+    f = lib.twq_fold_transforms
+    ws = lib.twq_fold_workspace_bytes(256, 128, 32)
+    assert ws >= 2 * 32 * 32 * 8 + 32 * 32 * 4 + 256 * 32 * 4
+    args = lambda **kw: [kw.get(k, d) for k, d in (
+        ("Q", A), ("G", A), ("U", A), ("V", A), ("R", A), ("m", 256), ("n", 128), ("r", 32),
+        ("L1", A), ("L2", A), ("Ro", A), ("ws", A), ("wsb", ws), ("st", None))]
+    assert f(*args(Q=None)) == 1
+    assert f(*args(m=0)) == 1
+    assert f(*args(r=1025)) == 2
+    assert f(*args(ws=A + 16)) == 3          # workspace must be 256-byte aligned
+    assert f(*args(wsb=ws - 1)) == 1
+    assert lib.twq_fold_workspace_bytes(0, 1, 1) == 0
+
+
 def test_lowrank_needs_rank(lib):
     w = _w(r=0)
     assert lib.twq_lowrank_only(A, A, 4, ctypes.byref(w), A, None) == 1
@@ -152,6 +167,7 @@ def test_launch_accounting(lib):
     assert twq.launches_per_call("twq_unfused_linear") == 4
     assert twq.launches_per_call("twq_unfused_linear_noalloc") == 4
     assert twq.launches_per_call("twq_fused_linear_x") == 1
+    assert twq.launches_per_call("twq_fold_transforms") == 5
     assert twq.launches_per_call("nope") == -1
 
 

@@ -23,6 +23,7 @@ enum WaitSite : int {
   kSiteDrainScaleFull = 9,
   kSiteFinal = 10,
   kSiteProducerHbFree = 11,
+  kSiteDrainPeerFree = 12,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -240,6 +241,13 @@ __device__ __forceinline__ void st_async_peer_v4(uint32_t raddr, float a, float 
       "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
       : "memory");
 }
+__device__ __forceinline__ void st_async_peer_v4u(uint32_t raddr, uint4 v, uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+          raddr),
+      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(rbar)
+      : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_peer(uint32_t raddr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(raddr)
                : "memory");
@@ -260,6 +268,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 __device__ __forceinline__ void cluster_sync_startup() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
+}
+// The two halves of the rendezvous, for kernels where only some warps touch
+// peer shared memory: every thread arrives once; a warp that goes on to write
+// into a peer (or arrive on a peer's barrier) waits before its first such access.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Shared-memory matrix descriptor, K-major operand in the 128-byte swizzle

@@ -253,10 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* rfull = bars;                     // [kMaxGroups] TMA of R tiles
   uint64_t* lfull = rfull + kMaxGroups;       // [kMaxGroups] TMA of L1 tiles
   uint64_t* al_full = lfull + kMaxGroups;     // [kRing] L1 operand slot written
-  uint64_t* al_empty = al_full + kRing;       // [kRing] L1 operand slot read by the MMA
-  uint64_t* ar_full = al_empty + kRing;       // [kRing] R operand slot written
-  uint64_t* ar_empty = ar_full + kRing;       // [kRing]
-  uint64_t* h_full = ar_empty + kRing;        // [kMaxGroups] stage-1 accumulator ready
+  // A ring slot is free again once the MMAs of the group that used it have completed,
+  // which is what that group's accumulator barrier (h_full / res_full) records: one
+  // tcgen05.commit per group serves both the drain and the next unpack into the slot.
+  uint64_t* ar_full = al_full + kRing;        // [kRing] R operand slot written
+  uint64_t* h_full = ar_full + kRing;         // [kMaxGroups] stage-1 accumulator ready
   uint64_t* res_full = h_full + kMaxGroups;   // [kMaxGroups] residual accumulator ready
   uint64_t* xfull = res_full + kMaxGroups;
   uint64_t* xready = xfull + 1;               // [kMaxGroups] group's X codes and scales ready
@@ -269,6 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
   volatile int* abort_flag = &s_abort;
 
+  // The next kernel on the stream may be scheduled now: its prologue and weight
+  // loads overlap this grid, and it reads this grid's output only after its
+  // griddepcontrol.wait, which waits for this grid to complete.
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int ks = static_cast<int>(cluster_rank());
@@ -300,9 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane < kRing) {
       mbar_init(&al_full[lane], 4);
-      mbar_init(&al_empty[lane], 1);
       mbar_init(&ar_full[lane], 4);
-      mbar_init(&ar_empty[lane], 1);
     }
     if (lane == 31) {
       mbar_init(xfull, 1);
@@ -341,19 +344,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(l2full, 16384);
         tma_load_2d(l2s, &tm_l2t, l2full, u0 * 16, n0);
       }
-      // The activations may come from the kernel just before this one on the
-      // stream (launched with programmatic serialization): wait for it first.
-      pdl_wait();
-      if (kQ) {  // BF16 X: two boxes of 64 elements x 16 tokens per group
-        mbar_arrive_expect_tx(xfull, ng * 4096);
-        for (int gi = 0; gi < ng; ++gi) {
-          tma_load_2d(xp + gi * 4096, &tm_xq, xfull, (g0 + gi) * 128, 0);
-          tma_load_2d(xp + gi * 4096 + 2048, &tm_xq, xfull, (g0 + gi) * 128 + 64, 0);
-        }
-      } else {
-        mbar_arrive_expect_tx(xfull, ng * 1024);
-        for (int gi = 0; gi < ng; ++gi) tma_load_2d(xp + gi * 1024, &tm_xq, xfull, (g0 + gi) * 64, 0);
-      }
     }
   }
   if (warp == 1) {
@@ -362,20 +352,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  // Every CTA of the cluster has initialized its barriers before any peer
-  // writes into its shared memory or arrives on its barriers.
-  cluster_sync_startup();
+  // Cluster rendezvous, split: every thread arrives here, after this CTA's barriers
+  // are initialized; only the exchange warps (12-19), the ones that store into peers'
+  // shared memory, wait for the peers' arrivals, just before their first push.
+  cluster_arrive_release();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+
+  // Everything above overlaps the preceding kernel on the stream (programmatic
+  // serialization). The activations may come from that kernel, so they are read
+  // only after griddepcontrol.wait; so that no bounded wait below counts the
+  // preceding kernel's run time, every role passes griddepcontrol.wait itself
+  // before its first wait that depends on X.
+  if (warp == 2 && lane == 0) {
+    pdl_wait();
+    if (kQ) {  // BF16 X: two boxes of 64 elements x 16 tokens per group
+      mbar_arrive_expect_tx(xfull, ng * 4096);
+      for (int gi = 0; gi < ng; ++gi) {
+        tma_load_2d(xp + gi * 4096, &tm_xq, xfull, (g0 + gi) * 128, 0);
+        tma_load_2d(xp + gi * 4096 + 2048, &tm_xq, xfull, (g0 + gi) * 128 + 64, 0);
+      }
+    } else {
+      mbar_arrive_expect_tx(xfull, ng * 1024);
+      for (int gi = 0; gi < ng; ++gi) tma_load_2d(xp + gi * 1024, &tm_xq, xfull, (g0 + gi) * 64, 0);
+    }
+  }
+  __syncwarp();
 
   if (kQ && (warp == 2 || warp == 3 || warp >= 12)) {
     // ----- X quantize (warps 2-3 and 12-19; 12-19 then go on to their own roles)
     const int qi = (warp < 4 ? warp - 2 : warp - 10) * 32 + lane;
+    pdl_wait();
     if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) quantize_slice(xp, ng, xu, sxs, xready, qi, lane);
   }
   if (warp == 0) {
     // ------------------------------------ residual MMA issuer (lane 0 of warp 0)
     if (lane == 0) {
+      pdl_wait();
       bool ok = true;
       const uint32_t xu0 = smem_u32(xu);
       const uint32_t idesc = idesc_i8(kNT);
@@ -391,7 +404,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 4; ++k)
             mma_i8_tmem_a(tmem_base + kColDres + gi * 16, tmem_base + kColR + slot * 32 + k * 8,
                           db + 2 * k, idesc, k > 0);
-          mma_commit(&ar_empty[slot]);
           mma_commit(&res_full[gi]);
         }
       }
@@ -409,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      pdl_wait();
       bool ok = true;
       const uint32_t xu0 = smem_u32(xu);
       const uint32_t idesc = idesc_i8(kNT);
@@ -424,7 +437,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 4; ++k)
             mma_i8_tmem_a(tmem_base + kColDh + gi * 16, tmem_base + kColL1 + slot * 32 + k * 8,
                           db + 2 * k, idesc, k > 0);
-          mma_commit(&al_empty[slot]);
           mma_commit(&h_full[gi]);
         }
       }
@@ -484,14 +496,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (is_l1 ? T::lr : T::res) {
       uint64_t* tfull = is_l1 ? lfull : rfull;
       uint64_t* sfull = is_l1 ? al_full : ar_full;
-      uint64_t* sempty = is_l1 ? al_empty : ar_empty;
+      uint64_t* done = is_l1 ? h_full : res_full;  // [gi]: the MMAs of group gi completed
       const uint8_t* tiles = is_l1 ? ltiles : rtiles;
       const int col0 = is_l1 ? kColL1 : kColR;
       for (int gi = 0; gi < ng; ++gi) {
         const int slot = gi % kRing;
-        const uint32_t ph = (gi / kRing) & 1;
         if (!d_wait<false>(&tfull[gi], 0, abort_flag, is_l1 ? kDSiteL1 : kDSiteR)) break;
-        if (!d_wait<false>(&sempty[slot], ph ^ 1u, abort_flag, is_l1 ? kDSiteAl : kDSiteAr)) break;
+        // the first kRing slots are free from the start; a later group takes the slot of
+        // group gi - kRing once that group's MMAs (which wait for X) have completed
+        if (gi >= kRing) {
+          if (gi == kRing) pdl_wait();
+          if (!d_wait<false>(&done[gi - kRing], 0, abort_flag, is_l1 ? kDSiteAl : kDSiteAr)) break;
+        }
         tc_fence_after();
         tile_row_to_tmem(tiles + gi * 8192, j, tmem_base + lane_addr + col0 + slot * 32);
         tmem_wait_st();
@@ -502,6 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 16) {
     // --------------- stage-1 drain, H exchange, BF16 H for stage 2 (warps 12-15)
+    cluster_wait_acquire();  // peers' barriers are initialized before the first push
+    pdl_wait();
     if (T::lr) {
       const int q = warp & 3;
       const int c = q * 32 + lane;  // index into r
@@ -574,6 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------- residual drain, Y exchange, store (warps 16-19)
+    cluster_wait_acquire();  // peers' barriers are initialized before the first push
+    pdl_wait();
     const int q = warp & 3;
     const int j = q * 32 + lane;  // column of the tile
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;

@@ -27,6 +27,8 @@
 // still pairs the same k and the per-group integer sums are unchanged.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "sm100_ptx.cuh"
 #include "twq_internal.h"
 
@@ -72,7 +74,7 @@ struct SmemLayout {
   static constexpr int kOffScale = kOffHb + kHb;
   static constexpr int kOffBar = kOffScale + kScaleSlots * kScaleSlot;
   static constexpr int kNumBars =
-      2 * kPackedStages + 2 * kUnpackedStages + 2 * kAccBufs + 2 * kScaleSlots + 3;
+      2 * kPackedStages + 2 * kUnpackedStages + 2 * kAccBufs + 2 * kScaleSlots + 4;
   static constexpr int kBytes = kOffBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
   static constexpr int kTmemCols = kAccBufs * BN;  // accumulator buffers
@@ -88,6 +90,7 @@ struct GemmArgs {
   int64_t b;
   int m, n, r, G;
   int row_blocks, col_tiles, num_tiles;
+  int tiles_per_rb;  // tiles (or, for CTA pairs, pairs of column tiles) per row block
   int r_pad;  // stage-2 K extent: r rounded up to 64
   int h_box;  // rows of the L1 TMA box: min(r, 128)
 };
@@ -133,6 +136,25 @@ __device__ __forceinline__ bool wait_fast(uint64_t* bar, uint32_t parity, volati
                                           int site) {
   if (mbar_try_wait(bar, parity)) return true;
   return wait_bar(bar, parity, abort_flag, site);
+}
+
+// Bounded wait with cluster-scope acquire, for barriers that complete on a peer
+// CTA's arrivals or stores.
+__device__ __noinline__ bool wait_bar_cluster(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int site) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      record_failure(site);
+      *abort_flag = 1;
+      return false;
+    }
+  }
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -244,15 +266,21 @@ struct TileInfo {
   bool need_h;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, int t, int t_begin, bool has_h) {
+// Work item t of a CTA's run: a tile, or for a CTA pair a pair of adjacent
+// column tiles of one row block, of which CTA `prank` takes one.
+__device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, int t, int t_begin, bool has_h,
+                                              int pair_stride, int prank) {
   TileInfo ti;
-  ti.rb = t / a.col_tiles;
-  ti.ct = t % a.col_tiles;
-  ti.need_h = has_h && (t == t_begin || (t - 1) / a.col_tiles != ti.rb);
+  ti.rb = t / a.tiles_per_rb;
+  ti.ct = (t % a.tiles_per_rb) * pair_stride + prank;
+  ti.need_h = has_h && (t == t_begin || (t - 1) / a.tiles_per_rb != ti.rb);
   return ti;
 }
 
-template <int kMode, int BN>
+// kPair: a cluster of two CTAs works on the two column tiles of one pair at a
+// time; CTA k computes H columns [k r/2, (k+1) r/2) of the row block and stores
+// its BF16 slice into both CTAs' H operand tiles, so H is computed once per pair.
+template <int kMode, int BN, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     twq_gemm_kernel(const __grid_constant__ CUtensorMap tm_xq,
                     const __grid_constant__ CUtensorMap tm_rq,
@@ -280,13 +308,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* hb_ready = sc_empty + kScaleSlots;
   uint64_t* hb_free = hb_ready + 1;
   uint64_t* mma_done = hb_free + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* peer_free = mma_done + 1;  // kPair: the peer may overwrite its slice of our H
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
   volatile int* abort_flag = &s_abort;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = args.G;
-  const int HC = T::h ? (args.r + kHChunk - 1) / kHChunk : 0;
+  // H chunks this CTA computes per row block: r in chunks of 128, or for a pair
+  // one chunk of r/2 columns at row offset prank * r/2 of L1
+  const int prank = kPair ? static_cast<int>(cluster_rank()) : 0;
+  const int HC = !T::h ? 0 : (kPair ? 1 : (args.r + kHChunk - 1) / kHChunk);
+  auto h_row0 = [&](int hc) { return kPair ? prank * (args.r / 2) : hc * kHChunk; };
+  auto h_cols = [&](int hc) { return kPair ? args.r / 2 : min(kHChunk, args.r - hc * kHChunk); };
   const int KC = args.r_pad / 64;
 
   if (threadIdx.x == 0) {
@@ -309,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(hb_ready, T::h_global ? 1 : 8);
     mbar_init(hb_free, 1);
     mbar_init(mma_done, 1);
+    mbar_init(peer_free, 1);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -339,8 +374,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int t_begin = static_cast<int>((int64_t)blockIdx.x * args.num_tiles / gridDim.x);
-  const int t_end = static_cast<int>((int64_t)(blockIdx.x + 1) * args.num_tiles / gridDim.x);
+  // Runs of work items: per CTA, or per CTA pair (both CTAs of a pair take the same run).
+  const int unit = kPair ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int units = kPair ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
+  const int t_begin = static_cast<int>((int64_t)unit * args.num_tiles / units);
+  const int t_end = static_cast<int>((int64_t)(unit + 1) * args.num_tiles / units);
+  constexpr int kPairStride = kPair ? 2 : 1;
+  // The peer's barriers are initialized before any remote store or arrive.
+  if (kPair) cluster_sync_startup();
 
   if (warp == 0) {
     // ------------------------------------------------------------- producer
@@ -354,19 +395,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t spend_phase[kScaleSlots];
       bool ok = true;
       for (int t = t_begin; t < t_end && ok; ++t) {
-        const TileInfo ti = tile_info(args, t, t_begin, T::h);
+        const TileInfo ti = tile_info(args, t, t_begin, T::h, kPairStride, prank);
         const int row0 = ti.rb * kBM;
         const int n0 = ti.ct * BN;
         if (ti.need_h) {
           for (int hc = 0; hc < HC && ok; ++hc) {
-            const int nh = min(kHChunk, args.r - hc * kHChunk);
+            const int nh = h_cols(hc);
             for (int g = 0; g < G; ++g) {
               if (!(ok = wait_fast(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
                 break;
               uint8_t* slot = slots + s.idx * L::kSlot;
               mbar_arrive_expect_tx(&full[s.idx], L::kSlotA + args.h_box * 64);
               tma_load_2d(slot, &tm_xq, &full[s.idx], g * 64, row0);
-              tma_load_2d(slot + L::kSlotA, &tm_l1q, &full[s.idx], g * 64, hc * kHChunk);
+              tma_load_2d(slot + L::kSlotA, &tm_l1q, &full[s.idx], g * 64, h_row0(hc));
               pend[s.idx] = true;
               pend_phase[s.idx] = s.phase;
               s.next(kPackedStages);
@@ -374,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   kSiteProducerScaleEmpty)))
                 break;
               mbar_arrive_expect_tx(&sc_full[q.idx], nh * 4);
-              bulk_load(scl + q.idx * BN, args.sl1 + (int64_t)g * args.r + hc * kHChunk, nh * 4,
+              bulk_load(scl + q.idx * BN, args.sl1 + (int64_t)g * args.r + h_row0(hc), nh * 4,
                         &sc_full[q.idx]);
               spend[q.idx] = true;
               spend_phase[q.idx] = q.phase;
@@ -444,10 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ua0 = smem_u32(ustg);
       const uint32_t hb0 = smem_u32(hb);
       for (int t = t_begin; t < t_end && ok; ++t) {
-        const TileInfo ti = tile_info(args, t, t_begin, T::h);
+        const TileInfo ti = tile_info(args, t, t_begin, T::h, kPairStride, prank);
         if (ti.need_h) {
           for (int hc = 0; hc < HC && ok; ++hc) {
-            const int nh = min(kHChunk, args.r - hc * kHChunk);
+            const int nh = h_cols(hc);
             const uint32_t idesc = idesc_i8(nh);
             for (int g = 0; g < G; ++g) {
               if (!(ok = wait_fast(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
@@ -486,7 +527,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (T::s2 && ok) {
           if (ti.need_h || T::h_global) {
-            if (!(ok = wait_fast(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) break;
+            if (kPair) {
+              // half of H came from the peer's st.async stores
+              if (!(ok = wait_bar_cluster(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) break;
+              fence_proxy_async_smem();
+            } else if (!(ok = wait_fast(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) {
+              break;
+            }
             hb_phase ^= 1u;
           }
           if (!(ok = wait_fast(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
@@ -523,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Ring s, u;
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t) {
-      const TileInfo ti = tile_info(args, t, t_begin, T::h);
+      const TileInfo ti = tile_info(args, t, t_begin, T::h, kPairStride, prank);
       const int n_h = ti.need_h ? HC * G : 0;
       const int n_res = T::res ? G : 0;
       const int n_l2 = T::s2 ? KC : 0;
@@ -536,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int brows = BN;
           if (step < n_h) {
             const int hc = step / G;
-            brows = min(kHChunk, args.r - hc * kHChunk);
+            brows = h_cols(hc);
           }
           unpack_tile(src, dst, kBM, plan);
           unpack_tile(src + L::kSlotA, dst + L::kUA, brows, plan);
@@ -561,17 +608,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_in = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     Ring a, q;
+    uint32_t peer_phase = 0;  // kPair: phase of peer_free for the next H slice
     bool ok = true;
     float acc[64];
     for (int t = t_begin; t < t_end && ok; ++t) {
-      const TileInfo ti = tile_info(args, t, t_begin, T::h);
+      const TileInfo ti = tile_info(args, t, t_begin, T::h, kPairStride, prank);
       const int64_t row = static_cast<int64_t>(ti.rb) * kBM + row_in;
       const bool row_ok = row < args.b;
       const float* sx_row = args.sx + (row_ok ? row : 0) * G;
       const int n0 = ti.ct * BN;
       if (ti.need_h) {
         for (int hc = 0; hc < HC && ok; ++hc) {
-          const int nh = min(kHChunk, args.r - hc * kHChunk);
+          const int nh = h_cols(hc);
           const int ncols = nh / 2;
           const int c0 = half * ncols;
 #pragma unroll
@@ -583,6 +631,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             sx0 = sx1;
             sx1 = (row_ok && g + 2 < G) ? __ldg(sx_row + g + 2) : 0.0f;
             if (!(ok = wait_bar(&acc_full[a.idx], a.phase, abort_flag, kSiteDrainAccFull))) break;
+            // The first stage-1 accumulator of a row block implies that every earlier MMA of
+            // this CTA, stage 2 of the previous row block included, has completed: the peer
+            // may now overwrite its slice of our H tile.
+            if (kPair && hc == 0 && g == 0 && dw == 0 && lane == 0)
+              mbar_arrive_peer(map_peer(smem_u32(peer_free), static_cast<uint32_t>(prank ^ 1)));
             tc_fence_after();
             if (!(ok = wait_bar(&sc_full[q.idx], q.phase, abort_flag, kSiteDrainScaleFull))) break;
             drain_group(acc, tmem_base + lane_addr + a.idx * BN + c0, ncols, scl + q.idx * BN + c0,
@@ -597,6 +650,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             q.next(kScaleSlots);
           }
           if (!ok) break;
+          // A pair stores its slice into the peer's H tile too, once the peer's stage 2 no
+          // longer reads it.
+          if (kPair) {
+            if (!(ok = wait_bar_cluster(peer_free, peer_phase, abort_flag, kSiteDrainPeerFree)))
+              break;
+            peer_phase ^= 1u;
+          }
           // H chunk complete: 2^-8 undoes the 16x16 code scaling of the unpack.
 #pragma unroll
           for (int j = 0; j < 64; j += 8) {
@@ -606,14 +666,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               o.y = pack_bf16x2(acc[j + 2] * 0.00390625f, acc[j + 3] * 0.00390625f);
               o.z = pack_bf16x2(acc[j + 4] * 0.00390625f, acc[j + 5] * 0.00390625f);
               o.w = pack_bf16x2(acc[j + 6] * 0.00390625f, acc[j + 7] * 0.00390625f);
-              const int col = hc * kHChunk + c0 + j;
+              const int col = h_row0(hc) + c0 + j;
               if (T::out_h) {
                 if (row_ok)
                   *reinterpret_cast<uint4*>(static_cast<uint16_t*>(args.out) + row * args.r +
                                             col) = o;
               } else {
-                *reinterpret_cast<uint4*>(hb + (col >> 6) * 16384 +
-                                          sw128_offset(row_in, (col & 63) >> 3)) = o;
+                uint8_t* dst = hb + (col >> 6) * 16384 + sw128_offset(row_in, (col & 63) >> 3);
+                *reinterpret_cast<uint4*>(dst) = o;
+                if (kPair) {
+                  const uint32_t peer = static_cast<uint32_t>(prank ^ 1);
+                  st_async_peer_v4u(map_peer(smem_u32(dst), peer), o,
+                                    map_peer(smem_u32(hb_ready), peer));
+                }
               }
             }
           }
@@ -622,7 +687,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!T::out_h) {
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(hb_ready);
+          if (lane == 0) {
+            // For a pair, one arrival also registers the bytes the peer stores into our
+            // H tile (its r/2 columns of the 128 rows, BF16).
+            if (kPair && dw == 0)
+              mbar_arrive_expect_tx(hb_ready, static_cast<uint32_t>(kBM * (args.r / 2) * 2));
+            else
+              mbar_arrive(hb_ready);
+          }
         }
       }
       if (T::out_h) continue;
@@ -718,6 +790,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
+  // A CTA of a pair leaves only after its peer is done: no store or arrive from the
+  // peer can still be on its way into this CTA's shared memory.
+  if (kPair) cluster_sync_startup();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
@@ -765,6 +840,40 @@ int num_sms() {
   return n > 0 ? n : 1;
 }
 
+// Clusters of two CTAs of the pair kernel that fit on the device at once, once
+// per instantiation (0 if the query fails: no pairs then).
+template <int kMode, int BN>
+int resident_pairs() {
+  static int cached = -1;
+  if (cached < 0) {
+    using L = SmemLayout<BN>;
+    auto kern = twq_gemm_kernel<kMode, BN, true>;
+    int nc = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = L::kAlloc;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();  // the query's own error: pairs are simply not used
+        nc = 0;
+      }
+    } else {
+      (void)cudaGetLastError();
+    }
+    cached = nc > 0 ? nc : 0;
+  }
+  return cached;
+}
+
 template <int kMode, int BN>
 cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
   using L = SmemLayout<BN>;
@@ -782,9 +891,30 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
   a.G = a.m / 128;
   a.row_blocks = static_cast<int>((c.b + kBM - 1) / kBM);
   a.col_tiles = T::out_h ? 1 : a.n / BN;
-  a.num_tiles = a.row_blocks * a.col_tiles;
+  // CTA pairs share H: modes with an on-chip H and stage 2, an even number of
+  // column tiles, and 128 < r <= 256 in two halves of whole 16-column MMA units.
+  // A step costs about the same at any MMA width up to 128, so halving H's columns
+  // pays only where it halves a CTA's H steps (two 128-wide chunks become one), and
+  // only where that saves more than the SMs that pairs leave idle (clusters are
+  // placed within a GPC): the choice compares the K-group steps of the busiest CTA.
+  bool pair = false;
+  if constexpr (T::h && T::s2 && !T::h_global) {
+    if (a.col_tiles % 2 == 0 && a.r % 32 == 0 && a.r > kHChunk && a.r <= 2 * kHChunk) {
+      const int pairs = resident_pairs<kMode, BN>();
+      const int hc1 = (a.r + kHChunk - 1) / kHChunk;
+      const int kc = (a.r + 63) / 64;
+      const int n1 = a.row_blocks * a.col_tiles, n2 = a.row_blocks * (a.col_tiles / 2);
+      const double t1 = static_cast<double>(n1) / std::min(n1, num_sms());
+      const double t2 = static_cast<double>(n2) / std::min(n2, pairs);
+      const double s1 = t1 * (a.G + kc) + (1.0 + t1 / a.col_tiles) * hc1 * a.G;
+      const double s2 = t2 * (a.G + kc) + (1.0 + t2 / (a.col_tiles / 2)) * a.G;
+      pair = pairs > 0 && s2 < 0.98 * s1;
+    }
+  }
+  a.tiles_per_rb = pair ? a.col_tiles / 2 : a.col_tiles;
+  a.num_tiles = a.row_blocks * a.tiles_per_rb;
   a.r_pad = ((a.r + 63) / 64) * 64;
-  a.h_box = a.r < kHChunk ? a.r : kHChunk;
+  a.h_box = pair ? a.r / 2 : (a.r < kHChunk ? a.r : kHChunk);
 
   CUtensorMap m_xq{}, m_rq{}, m_l1q{}, m_l2t{}, m_h{};
   const uint64_t kb = static_cast<uint64_t>(a.m / 2);
@@ -804,12 +934,41 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
                          static_cast<uint64_t>(a.r) * 2, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
 
-  auto kern = twq_gemm_kernel<kMode, BN>;
+  if (!pair || !(T::h && T::s2 && !T::h_global)) {
+    auto kern = twq_gemm_kernel<kMode, BN, false>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
+    kern<<<grid, kThreads, L::kAlloc, st>>>(m_xq, m_rq, m_l1q, m_l2t, m_h, a);
+    return cudaGetLastError();
+  }
+  if constexpr (T::h && T::s2 && !T::h_global) {
+  auto kern = twq_gemm_kernel<kMode, BN, true>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  int grid = a.num_tiles < num_sms() ? a.num_tiles : num_sms();
-  kern<<<grid, kThreads, L::kAlloc, st>>>(m_xq, m_rq, m_l1q, m_l2t, m_h, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // One wave of persistent pairs: as many as can be resident at once.
+  const int rp = resident_pairs<kMode, BN>();
+  const int pairs = a.num_tiles < rp ? a.num_tiles : rp;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  e = cudaLaunchKernelEx(&cfg, kern, m_xq, m_rq, m_l1q, m_l2t, m_h, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+  } else {
+    return cudaErrorInvalidValue;  // unreachable: `pair` implies the condition above
+  }
 }
 
 }  // namespace

@@ -181,6 +181,9 @@ def test_pack_weights_bitexact(twq, device, name):
 SHAPES = [  # b, m, n, r: several tiles, ragged b, one/two H chunks, r not a multiple of 64
     (16, 512, 512, 32), (1, 128, 128, 16), (3, 256, 384, 48), (17, 384, 256, 64),
     (129, 512, 384, 128), (200, 256, 256, 144), (64, 640, 128, 256), (300, 128, 512, 16),
+    # CTA pairs sharing H (even column-tile count, 128 < r <= 256, r % 32 == 0): halves of
+    # r/2 = 112 and 80 that straddle 64-column chunks, three pair items per row block, r = 256
+    (129, 256, 512, 224), (200, 256, 256, 192), (257, 384, 768, 160), (300, 256, 1024, 256),
 ]
 
 

@@ -158,54 +158,71 @@ __device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int j, uin
 
 // Eq. (1) quantizer fused into the prologue. The CTA's BF16 slice of X sits in
 // shared memory as two TMA boxes per group (64 elements x 16 tokens each, rows
-// of 128 bytes; tokens >= b read as zero). Eight lanes take one (token, group)
-// pair, 16 elements each; quantizing lane `qi` of 80 (warps 2-3 and 12-19)
-// handles the pairs qi / 8 + 10 k. Codes go to the 128-byte-swizzle B tiles as
-// 16*q in the in-chunk order of unpack8, scales to sxs, with the arithmetic of
-// twq_quantize_act, so the codes are identical.
-constexpr int kQPairsPerPass = 40;  // 10 warps x 4 pairs
+// of 128 bytes; tokens >= b read as zero). Four lanes take one (token, group)
+// pair: lane l of the four covers the 16-element chunks l and l + 4 (elements
+// [16 l, 16 l + 16) of each box). Quantizing lane `qi` of 320 (warps 2-3 and
+// 12-19) handles the pairs qi / 4 + 80 k, so the 128 pairs of eight groups take
+// two passes. Codes go to the 128-byte-swizzle B tiles as 16*q in the in-chunk
+// order of unpack8, scales to sxs, with the arithmetic of twq_quantize_act, so
+// the codes are identical (the group maximum is exact in any order).
+constexpr int kQPairsPerPass = 80;  // 10 warps x 8 pairs
+
+__device__ __forceinline__ uint4 pack_codes16(const uint32_t (&nb)[16]) {
+  // 16*q bytes: even elements 0..6, odd 1..7, even 8..14, odd 9..15
+  uint4 o;
+  o.x = (nb[0] << 4) | (nb[1] << 12) | (nb[2] << 20) | (nb[3] << 28);
+  o.y = (nb[8] << 4) | (nb[9] << 12) | (nb[10] << 20) | (nb[11] << 28);
+  o.z = (nb[4] << 4) | (nb[5] << 12) | (nb[6] << 20) | (nb[7] << 28);
+  o.w = (nb[12] << 4) | (nb[13] << 12) | (nb[14] << 20) | (nb[15] << 28);
+  return o;
+}
 
 __device__ __forceinline__ void quantize_slice(const uint8_t* xs, int ng, uint8_t* xu, float* sxs,
                                                uint64_t* xready, int qi, int lane) {
-  const int l = lane & 7;  // elements [16 l, 16 l + 16) of the group
+  const int l = lane & 3;
   const int pairs = kNT * ng;
   const int passes = (pairs + kQPairsPerPass - 1) / kQPairsPerPass;  // uniform over the warp
 #pragma unroll 1
   for (int it = 0; it < passes; ++it) {
-    const int p = (qi >> 3) + it * kQPairsPerPass;
+    const int p = (qi >> 2) + it * kQPairsPerPass;
     const bool pv = p < pairs;
     const int gi = pv ? p / kNT : 0, t = pv ? p % kNT : 0;
-    const uint8_t* src = xs + gi * 4096 + (l >> 2) * 2048 + t * 128 + (l & 3) * 32;
-    const uint4 r0 = *reinterpret_cast<const uint4*>(src);
-    const uint4 r1 = *reinterpret_cast<const uint4*>(src + 16);
-    const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-    // f[0..7]: even elements 0, 2, .., 14 of the lane's 16; f[8..15]: odd elements
-    float f[16];
+    const uint8_t* src = xs + gi * 4096 + t * 128 + l * 32;
+    // f[h][0..7]: even elements 0, 2, .., 14 of chunk l + 4h; f[h][8..15]: odd elements
+    float f[2][16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f[i] = __uint_as_float(w[i] << 16);
-      f[8 + i] = __uint_as_float(w[i] & 0xFFFF0000u);
+    for (int h = 0; h < 2; ++h) {
+      const uint4 r0 = *reinterpret_cast<const uint4*>(src + h * 2048);
+      const uint4 r1 = *reinterpret_cast<const uint4*>(src + h * 2048 + 16);
+      const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        f[h][i] = __uint_as_float(w[i] << 16);
+        f[h][8 + i] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
     }
     float m4[4];  // absmax as a tree, for instruction-level parallelism
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      m4[i] = fmaxf(fmaxf(fabsf(f[i]), fabsf(f[i + 4])), fmaxf(fabsf(f[i + 8]), fabsf(f[i + 12])));
+      m4[i] = fmaxf(fmaxf(fmaxf(fabsf(f[0][i]), fabsf(f[0][i + 4])),
+                          fmaxf(fabsf(f[0][i + 8]), fabsf(f[0][i + 12]))),
+                    fmaxf(fmaxf(fabsf(f[1][i]), fabsf(f[1][i + 4])),
+                          fmaxf(fabsf(f[1][i + 8]), fabsf(f[1][i + 12]))));
     float a = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 #pragma unroll
-    for (int off = 4; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+    for (int off = 2; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
     const Eq1Scale ks = eq1_scale(a);
-    uint4 o = make_uint4(0, 0, 0, 0);
+    uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
     if (ks.s != 0.0f) {
       uint32_t nb[16];
-      eq1_nibbles(f, ks, nb);
-      // 16*q bytes: even elements 0..6, odd 1..7, even 8..14, odd 9..15
-      o.x = (nb[0] << 4) | (nb[1] << 12) | (nb[2] << 20) | (nb[3] << 28);
-      o.y = (nb[8] << 4) | (nb[9] << 12) | (nb[10] << 20) | (nb[11] << 28);
-      o.z = (nb[4] << 4) | (nb[5] << 12) | (nb[6] << 20) | (nb[7] << 28);
-      o.w = (nb[12] << 4) | (nb[13] << 12) | (nb[14] << 20) | (nb[15] << 28);
+      eq1_nibbles(f[0], ks, nb);
+      o0 = pack_codes16(nb);
+      eq1_nibbles(f[1], ks, nb);
+      o1 = pack_codes16(nb);
     }
     if (pv) {
-      *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(t, l)) = o;
+      *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(t, l)) = o0;
+      *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(t, l + 4)) = o1;
       if (l == 0) sxs[gi * kNT + t] = ks.s;
     }
     // Groups whose last pair falls in this pass are complete once every warp
@@ -647,14 +664,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     int keep_waiting = 0;  // not the abort flag: peers may still be writing into this CTA
     const bool got = d_wait<true>(y_ready, 0, &keep_waiting, kDSiteYReady);
     if (ok && got) {
+      // A thread sums four consecutive tokens of one column (16-byte reads: a quarter
+      // warp reads 128 contiguous bytes, so the loads are free of bank conflicts),
+      // over the ranks in order.
       const int tid = threadIdx.x - 512;
-      for (int e = tid; e < kColsPerOwner * kNT; e += 128) {
-        const int t = e / kColsPerOwner, jl = e % kColsPerOwner;
-        float yv = 0.0f;
-        for (int k = 0; k < KS; ++k) yv += yred[(k * kColsPerOwner + jl) * kNT + t];
-        if (t < args.b)
-          args.y[static_cast<int64_t>(t) * args.n + n0 + ks * kColsPerOwner + jl] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(yv));
+      for (int e = tid; e < kColsPerOwner * (kNT / 4); e += 128) {
+        const int tc = e & 3, jl = e >> 2;
+        float yv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int k = 0; k < KS; ++k) {
+          const float4 v = *reinterpret_cast<const float4*>(yred + (k * kColsPerOwner + jl) * kNT + tc * 4);
+          yv[0] += v.x;
+          yv[1] += v.y;
+          yv[2] += v.z;
+          yv[3] += v.w;
+        }
+        uint16_t* yc = args.y + n0 + ks * kColsPerOwner + jl;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = tc * 4 + i;
+          if (t < args.b)
+            yc[static_cast<int64_t>(t) * args.n] = __bfloat16_as_ushort(__float2bfloat16_rn(yv[i]));
+        }
       }
     }
   }

@@ -453,18 +453,27 @@ def run_e2e(prob, K, W, world, device):
     import torch
     from rank_residual_w4a4_b200 import twq
     xh = torch.from_numpy(prob.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-    yh = torch.empty((prob.b, prob.n), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(prob.x[0])
+    # Decode steps rotate over four streams, each with its own device and pinned host
+    # buffers, so a step's copies (about 6 us each way for 128 KB) overlap the other
+    # streams' layer kernels; with fewer streams the per-stream chain H2D -> layer ->
+    # D2H sets the pace.
+    streams = [torch.cuda.Stream(device) for _ in range(4)]
+    xds = [torch.empty_like(prob.x[0]) for _ in streams]
+    yds = [torch.empty_like(prob.y[0]) for _ in streams]
+    yhs = [torch.empty((prob.b, prob.n), dtype=torch.bfloat16).pin_memory() for _ in streams]
+    steps = ([twq.DecodeStep(xds[j], yds[j], yhs[j], stream=streams[j]) for j in range(len(streams))]
+             if prob.one_launch else None)
 
     def one(i):
         c = i % prob.copies
-        xd.copy_(xh, non_blocking=True)
         if prob.one_launch:
-            y = twq.fused_linear_x(xd, prob.weights[c], prob.y[c])
+            steps[i % len(steps)](xh, prob.weights[c])
         else:
+            xd = xds[0]
+            xd.copy_(xh, non_blocking=True)
             xq, sx = twq.quantize_act(xd, prob.xq[c], prob.sx[c])
             y = twq.fused_linear(xq, sx, prob.weights[c], prob.y[c])
-        yh.copy_(y, non_blocking=True)
+            yhs[0].copy_(y, non_blocking=True)
 
     for i in range(W):
         one(i)
@@ -472,16 +481,26 @@ def run_e2e(prob, K, W, world, device):
     barrier(world)
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
-    s.record()
+    cur = torch.cuda.current_stream()
+    s.record(cur)
+    for st in streams:  # the steps' streams start after s ...
+        st.wait_event(s)
+    h0 = time.perf_counter()
     for i in range(K):
         one(i)
-    e.record()
+    host_s = time.perf_counter() - h0  # host time to issue the K steps
+    for st in streams:  # ... and e waits for both of them
+        cur.wait_stream(st)
+    e.record(cur)
     torch.cuda.synchronize()
     barrier(world)
     t = max_over_ranks(s.elapsed_time(e) / 1e3, world, device)
     return {"value": round(prob.b * world * K / t, 1), "unit": "tokens/s",
             "h2d_bytes_per_step": prob.b * prob.m * 2, "d2h_bytes_per_step": prob.b * prob.n * 2,
-            "path": "python binding, eager launches"}
+            "host_issue_us_per_step": round(host_s / K * 1e6, 2),
+            "path": ("twq.DecodeStep -> twq_fused_linear_x_host (H2D, layer, D2H in one C-ABI "
+                     "call), eager, four streams in rotation" if prob.one_launch else
+                     "python binding, eager launches")}
 
 
 def sweep(args, device, peaks):

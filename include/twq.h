@@ -137,7 +137,10 @@ TWQ_API twq_status twq_pack_weights(const uint16_t* R, const uint16_t* L1, const
  * reads of the packed weights start while that kernel is still running, and
  * its reads of xq / sx wait until that kernel has completed. So xq / sx may come
  * from the preceding kernel, but the weights must not be written by a kernel
- * that signals early (twq_pack_weights does not).
+ * that signals early (twq_pack_weights does not). The decode kernel itself
+ * signals at entry, so the next decode call's prologue and weight reads overlap
+ * it; a kernel of the caller's that is launched after it with programmatic
+ * serialization must wait (griddepcontrol.wait) before it reads y.
  */
 TWQ_API twq_status twq_fused_linear(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
                             uint16_t* y, twq_stream_t stream);
@@ -159,6 +162,26 @@ TWQ_API twq_status twq_fused_linear(const uint8_t* xq, const float* sx, int64_t 
  */
 TWQ_API twq_status twq_fused_linear_x(const uint16_t* x, int64_t ldx, int64_t b,
                                       const twq_weights* w, uint16_t* y, twq_stream_t stream);
+
+/*
+ * twq_fused_linear_x from host memory to host memory (TwinQuant §4.3, one decode
+ * step of the layer as a serving loop issues it). On `stream`, in order:
+ *   1. copy x_host (b x m BF16, row-major, contiguous) into x_dev;
+ *   2. run twq_fused_linear_x on x_dev (ldx = m), writing y_dev (b x n BF16);
+ *   3. copy y_dev into y_host (b x n BF16, row-major, contiguous).
+ * Nothing is synchronized: the call returns once the three operations are
+ * enqueued, and y_host holds the result once the stream reaches that point (an
+ * event or a stream synchronize). Host buffers should be page-locked
+ * (cudaHostAlloc / cudaHostRegister), or the copies are not asynchronous. The
+ * caller owns all buffers; x_dev and y_dev must not be in use by other work on
+ * other streams while the step runs (a loop that overlaps steps on two streams
+ * gives each stream its own x_dev, y_dev and y_host).
+ * Limits and errors: those of twq_fused_linear_x, all checked before anything is
+ * enqueued; TWQ_ERR_CUDA if enqueueing a copy or the launch fails.
+ */
+TWQ_API twq_status twq_fused_linear_x_host(const uint16_t* x_host, int64_t b, const twq_weights* w,
+                                           uint16_t* x_dev, uint16_t* y_dev, uint16_t* y_host,
+                                           twq_stream_t stream);
 
 /* Residual component only: Y = bf16(Q(X) Q(R)) (TwinQuant Eq. (2)); ignores l1q/sl1/l2t. */
 TWQ_API twq_status twq_w4a4_only(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,

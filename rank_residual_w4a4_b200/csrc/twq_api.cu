@@ -146,13 +146,9 @@ twq_status twq_lowrank_only(const uint8_t* xq, const float* sx, int64_t b, const
   return run(twq::kModeLowRank, xq, sx, b, w, y, nullptr, stream);
 }
 
-twq_status twq_fused_linear_x(const uint16_t* x, int64_t ldx, int64_t b, const twq_weights* w,
-                              uint16_t* y, twq_stream_t stream) {
-  if (!w) return TWQ_ERR_INVALID_ARG;
-  twq_status s = shape_ok(w->m, w->n, w->r);
-  if (s != TWQ_OK) return s;
-  if (b < 0 || ldx < w->m) return TWQ_ERR_INVALID_ARG;
-  if (b == 0) return TWQ_OK;
+// Validates a twq_fused_linear_x call (b >= 1) and fills the decode launch.
+static twq_status prepare_fused_x(const uint16_t* x, int64_t ldx, int64_t b, const twq_weights* w,
+                                  uint16_t* y, twq::GemmCall* out) {
   if (!x || !y || !w->rq || !w->sr) return TWQ_ERR_INVALID_ARG;
   if (!aligned16(x) || ldx % 8 || !aligned16(y) || !aligned16(w->rq) || !aligned16(w->sr))
     return TWQ_ERR_MISALIGNED;
@@ -165,7 +161,42 @@ twq_status twq_fused_linear_x(const uint16_t* x, int64_t ldx, int64_t b, const t
   c.x = x;
   c.ldx = ldx;
   if (!twq::decode_eligible(c)) return TWQ_ERR_UNSUPPORTED;
+  *out = c;
+  return TWQ_OK;
+}
+
+twq_status twq_fused_linear_x(const uint16_t* x, int64_t ldx, int64_t b, const twq_weights* w,
+                              uint16_t* y, twq_stream_t stream) {
+  if (!w) return TWQ_ERR_INVALID_ARG;
+  twq_status s = shape_ok(w->m, w->n, w->r);
+  if (s != TWQ_OK) return s;
+  if (b < 0 || ldx < w->m) return TWQ_ERR_INVALID_ARG;
+  if (b == 0) return TWQ_OK;
+  twq::GemmCall c{};
+  if ((s = prepare_fused_x(x, ldx, b, w, y, &c)) != TWQ_OK) return s;
   return from_cuda(twq::launch_decode(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+twq_status twq_fused_linear_x_host(const uint16_t* x_host, int64_t b, const twq_weights* w,
+                                   uint16_t* x_dev, uint16_t* y_dev, uint16_t* y_host,
+                                   twq_stream_t stream) {
+  if (!w) return TWQ_ERR_INVALID_ARG;
+  twq_status s = shape_ok(w->m, w->n, w->r);
+  if (s != TWQ_OK) return s;
+  if (b < 0) return TWQ_ERR_INVALID_ARG;
+  if (b == 0) return TWQ_OK;
+  if (!x_host || !y_host) return TWQ_ERR_INVALID_ARG;
+  twq::GemmCall c{};
+  if ((s = prepare_fused_x(x_dev, w->m, b, w, y_dev, &c)) != TWQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(b) * w->m * 2, yb = static_cast<size_t>(b) * w->n * 2;
+  if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return TWQ_ERR_CUDA;
+  cudaError_t e = twq::launch_decode(c, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return TWQ_ERR_CUDA;
+  return TWQ_OK;
 }
 
 size_t twq_unfused_workspace_bytes(int64_t b, int64_t n, int64_t r) {
@@ -215,7 +246,8 @@ int twq_launches_per_call(const char* ep) {
   if (!strcmp(ep, "twq_quantize_act")) return 1;
   if (!strcmp(ep, "twq_pack_weights")) return 3;
   if (!strcmp(ep, "twq_fused_linear") || !strcmp(ep, "twq_w4a4_only") ||
-      !strcmp(ep, "twq_lowrank_only") || !strcmp(ep, "twq_fused_linear_x"))
+      !strcmp(ep, "twq_lowrank_only") || !strcmp(ep, "twq_fused_linear_x") ||
+      !strcmp(ep, "twq_fused_linear_x_host"))
     return 1;
   if (!strcmp(ep, "twq_unfused_linear") || !strcmp(ep, "twq_unfused_linear_noalloc")) return 4;
   if (!strcmp(ep, "twq_fold_transforms")) return 5;

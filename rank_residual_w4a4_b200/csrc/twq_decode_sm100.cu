@@ -27,6 +27,7 @@
 // the exact byte count it expects before the cluster rendezvous). A CTA never
 // reads a peer's shared memory, and every write into it has landed once its
 // bounded wait completes, so no CTA exits while a peer may still write into it.
+#include <atomic>
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
@@ -757,9 +758,17 @@ cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
                         static_cast<uint64_t>(a.r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
   auto kern = twq_decode_kernel<kMode, KS, kQ>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DLayout::kAlloc);
+  // The shared-memory opt-in is a driver call: once per instantiation and device.
+  static std::atomic<uint64_t> smem_set{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (!bit || !(smem_set.load(std::memory_order_relaxed) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DLayout::kAlloc);
+    if (e != cudaSuccess) return e;
+    smem_set.fetch_or(bit);
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(KS, a.n / 128, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -27,7 +27,8 @@ EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_siz
            "twq_quantize_act", "twq_pack_weights", "twq_fused_linear", "twq_w4a4_only",
            "twq_lowrank_only", "twq_unfused_workspace_bytes", "twq_unfused_linear",
            "twq_device_status", "twq_launches_per_call", "twq_unfused_linear_noalloc",
-           "twq_fused_linear_x", "twq_fold_workspace_bytes", "twq_fold_transforms")
+           "twq_fused_linear_x", "twq_fold_workspace_bytes", "twq_fold_transforms",
+           "twq_fused_linear_x_host")
 
 
 class TwqError(RuntimeError):
@@ -71,6 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twq_launches_per_call": ([ctypes.c_char_p], ctypes.c_int),
         "twq_unfused_linear_noalloc": ([P, P, I, P, P, P], ctypes.c_int),
         "twq_fused_linear_x": ([P, I, I, P, P, P], ctypes.c_int),
+        "twq_fused_linear_x_host": ([P, I, P, P, P, P, P], ctypes.c_int),
         "twq_fold_workspace_bytes": ([I, I, I], S),
         "twq_fold_transforms": ([P, P, P, P, P, I, I, I, P, P, P, P, S, P], ctypes.c_int),
     }
@@ -132,10 +134,21 @@ class Weights:
     sl1: torch.Tensor   # m/128 x r float32
     l2t: torch.Tensor   # n x r bfloat16
 
+    def __setattr__(self, name, value):
+        object.__setattr__(self, name, value)
+        if name != "_c":
+            object.__setattr__(self, "_c", None)  # a field changed: rebuild the C view
+
     def c_struct(self) -> _Weights:
-        nz = lambda t: t.data_ptr() if t.numel() else None
-        return _Weights(self.m, self.n, self.r, self.rq.data_ptr(), self.sr.data_ptr(),
-                        nz(self.l1q), nz(self.sl1), nz(self.l2t))
+        """The C-ABI view (built once; the library only reads it during a call). It
+        follows field reassignment, not a tensor re-pointed in place (Tensor.set_)."""
+        c = getattr(self, "_c", None)
+        if c is None:
+            nz = lambda t: t.data_ptr() if t.numel() else None
+            c = _Weights(self.m, self.n, self.r, self.rq.data_ptr(), self.sr.data_ptr(),
+                         nz(self.l1q), nz(self.sl1), nz(self.l2t))
+            object.__setattr__(self, "_c", c)
+        return c
 
     @staticmethod
     def empty(m: int, n: int, r: int, device) -> "Weights":
@@ -210,6 +223,63 @@ def fused_linear_x(x: torch.Tensor, w: Weights, y=None, stream=None):
                                      _dev(y, "y", torch.bfloat16), _stream(stream)),
            "twq_fused_linear_x")
     return y
+
+
+def fused_linear_x_host(x_host: torch.Tensor, w: Weights, x_dev: torch.Tensor,
+                        y_dev: torch.Tensor, y_host: torch.Tensor, stream=None):
+    """One decode step from host memory to host memory on `stream`: copy x_host into
+    x_dev, run fused_linear_x, copy y_dev into y_host. Nothing is synchronized; y_host
+    holds Y once the stream reaches the end of the step. Host tensors should be pinned."""
+    for t, name in ((x_host, "x_host"), (y_host, "y_host")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda:
+            raise TypeError("%s must be a host (CPU) torch tensor" % name)
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise TypeError("%s must be a contiguous torch.bfloat16 tensor" % name)
+    b = x_host.shape[0]
+    if x_host.shape != (b, w.m) or y_host.shape != (b, w.n):
+        raise ValueError("x_host must be (b, m) and y_host (b, n)")
+    if x_dev.shape != (b, w.m) or y_dev.shape != (b, w.n):
+        raise ValueError("x_dev must be (b, m) and y_dev (b, n)")
+    cw = w.c_struct()
+    _check(load().twq_fused_linear_x_host(x_host.data_ptr(), b, ctypes.byref(cw),
+                                          _dev(x_dev, "x_dev", torch.bfloat16),
+                                          _dev(y_dev, "y_dev", torch.bfloat16),
+                                          y_host.data_ptr(), _stream(stream)),
+           "twq_fused_linear_x_host")
+    return y_host
+
+
+class DecodeStep:
+    """A prepared twq_fused_linear_x_host call for a serving loop. The device
+    buffers, the pinned host output and the stream are checked once; each call
+    passes a host X of the same shape and the layer's weights (their C view is
+    cached on the Weights object), so a step costs one C call."""
+
+    def __init__(self, x_dev: torch.Tensor, y_dev: torch.Tensor, y_host: torch.Tensor, stream=None):
+        self._b, self._m = x_dev.shape
+        if y_dev.shape[0] != self._b or y_host.shape != y_dev.shape:
+            raise ValueError("x_dev (b, m), y_dev and y_host (b, n) must agree")
+        if not isinstance(y_host, torch.Tensor) or y_host.is_cuda:
+            raise TypeError("y_host must be a host (CPU) torch tensor")
+        if y_host.dtype != torch.bfloat16 or not y_host.is_contiguous():
+            raise TypeError("y_host must be a contiguous torch.bfloat16 tensor")
+        self._n = y_dev.shape[1]
+        self._xd = _dev(x_dev, "x_dev", torch.bfloat16)
+        self._yd = _dev(y_dev, "y_dev", torch.bfloat16)
+        self._yh = y_host.data_ptr()
+        self._keep = (x_dev, y_dev, y_host)  # the buffers outlive the prepared call
+        self._st = _stream(stream)
+        self._fn = load().twq_fused_linear_x_host
+        self.y_host = y_host
+
+    def __call__(self, x_host: torch.Tensor, w: Weights) -> torch.Tensor:
+        if x_host.is_cuda or x_host.dtype != torch.bfloat16 or not x_host.is_contiguous():
+            raise TypeError("x_host must be a contiguous host torch.bfloat16 tensor")
+        if x_host.shape[0] != self._b or x_host.shape[1] != self._m or w.m != self._m or w.n != self._n:
+            raise ValueError("x_host and w must match the prepared shapes")
+        _check(self._fn(x_host.data_ptr(), self._b, ctypes.byref(w.c_struct()), self._xd, self._yd,
+                        self._yh, self._st), "twq_fused_linear_x_host")
+        return self.y_host
 
 
 def fold_workspace_bytes(m: int, n: int, r: int) -> int:

@@ -125,6 +125,22 @@ def test_fused_linear_x_validation(lib):
     assert f(A, 512, 4, ctypes.byref(big), A, None) == 2
 
 
+def test_fused_linear_x_host_validation(lib):
+    # every rejection happens before anything is enqueued, so these run without a GPU
+    f = lib.twq_fused_linear_x_host
+    w = _w()
+    assert f(A, 4, None, A, A, A, None) == 1
+    assert f(None, 4, ctypes.byref(w), A, A, A, None) == 1   # no host X
+    assert f(A, 4, ctypes.byref(w), A, A, None, None) == 1   # no host Y
+    assert f(A, 4, ctypes.byref(w), None, A, A, None) == 1   # no device X
+    assert f(A, -1, ctypes.byref(w), A, A, A, None) == 1
+    assert f(A, 4, ctypes.byref(w), A + 2, A, A, None) == 3
+    assert f(A, 4, ctypes.byref(w), A, A + 4, A, None) == 3
+    assert f(None, 0, ctypes.byref(w), None, None, None, None) == 0   # b == 0: nothing to do
+    assert f(A, 17, ctypes.byref(w), A, A, A, None) == 2     # b > 16
+    assert f(A, 4, ctypes.byref(_w(r=144)), A, A, A, None) == 2
+
+
 def test_fold_validation(lib):
     f = lib.twq_fold_transforms
     ws = lib.twq_fold_workspace_bytes(256, 128, 32)
@@ -167,6 +183,7 @@ def test_launch_accounting(lib):
     assert twq.launches_per_call("twq_unfused_linear") == 4
     assert twq.launches_per_call("twq_unfused_linear_noalloc") == 4
     assert twq.launches_per_call("twq_fused_linear_x") == 1
+    assert twq.launches_per_call("twq_fused_linear_x_host") == 1
     assert twq.launches_per_call("twq_fold_transforms") == 5
     assert twq.launches_per_call("nope") == -1
 

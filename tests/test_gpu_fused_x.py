@@ -165,3 +165,45 @@ def test_fused_x_decode_workload(twq, device, b):
     assert np.array_equal(y, _two_call(twq, xd, w))
     assert_y_close(y, oracle.layer(x, R, L1, L2, mode=oracle.FUSED)["y"], "decode b=%d" % b)
     _status_clean(twq)
+
+
+@pytest.mark.parametrize("b,m,n,r", [(16, 4096, 512, 128), (3, 1024, 384, 48), (1, 2048, 256, 0)])
+def test_host_step_matches_device_call(twq, device, b, m, n, r):
+    """twq_fused_linear_x_host: host X in, host Y out, on two streams with their own
+    buffers; Y bitwise equal to twq_fused_linear_x on the device copy of X."""
+    import torch
+    x, R, L1, L2 = _operands(b, m, n, r, seed=31)
+    w = _pack(twq, device, R, L1, L2)
+    ref = bits_of(twq.fused_linear_x(to_dev(x, device), w))
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    streams = [torch.cuda.Stream(device), torch.cuda.Stream(device)]
+    bufs = [(torch.empty((b, m), dtype=torch.bfloat16, device=device),
+             torch.empty((b, n), dtype=torch.bfloat16, device=device),
+             torch.empty((b, n), dtype=torch.bfloat16).pin_memory()) for _ in streams]
+    for i in range(6):
+        xd, yd, yh = bufs[i % 2]
+        yh.fill_(0)
+        twq.fused_linear_x_host(xh, w, xd, yd, yh, stream=streams[i % 2])
+    torch.cuda.synchronize()
+    for _, _, yh in bufs:
+        assert np.array_equal(yh.view(torch.int16).numpy().view(np.uint16), ref)
+    _status_clean(twq)
+
+
+def test_prepared_decode_step(twq, device):
+    """twq.DecodeStep: the prepared form of the host call gives the same Y."""
+    import torch
+    b, m, n, r = 8, 2048, 384, 64
+    x, R, L1, L2 = _operands(b, m, n, r, seed=33)
+    w = _pack(twq, device, R, L1, L2)
+    ref = bits_of(twq.fused_linear_x(to_dev(x, device), w))
+    step = twq.DecodeStep(torch.empty((b, m), dtype=torch.bfloat16, device=device),
+                          torch.empty((b, n), dtype=torch.bfloat16, device=device),
+                          torch.zeros((b, n), dtype=torch.bfloat16).pin_memory())
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = step(xh, w)
+    torch.cuda.synchronize()
+    assert np.array_equal(yh.view(torch.int16).numpy().view(np.uint16), ref)
+    with pytest.raises(ValueError):
+        step(xh[: b - 1].contiguous(), w)
+    _status_clean(twq)

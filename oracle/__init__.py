@@ -46,6 +46,8 @@ def _get():
         lib = ctypes.CDLL(build())
         for name, args in {
             "twq_ref_quant_group_f32": [_P, ctypes.c_int, _P, _P],
+            "twq_ref_quant_group_f32_a8": [_P, ctypes.c_int, _P, _P],
+            "twq_ref_quantize_rows_q": [_P, _I, _I, _I, ctypes.c_int, _P, _P],
             "twq_ref_quantize_rows": [_P, _I, _I, _I, _P, _P],
             "twq_ref_quantize_cols": [_P, _I, _I, _P, _P],
             "twq_ref_pack_nibbles": [_P, _I, _P],
@@ -63,6 +65,7 @@ def _get():
         lib.twq_ref_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.twq_ref_f32_to_bf16.restype = ctypes.c_uint16
         lib.twq_ref_qmax.restype = ctypes.c_int
+        lib.twq_ref_qmax_a8.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -84,21 +87,29 @@ def qmax() -> int:
     return _get().twq_ref_qmax()
 
 
-def quant_group_f32(v):
+def qmax_a8() -> int:
+    """q_max of the W4A8 activations (Eq. (1) with k = 8)."""
+    return _get().twq_ref_qmax_a8()
+
+
+def quant_group_f32(v, a8=False):
     v = _c(v, np.float32)
     q = np.empty(v.size, np.int8)
     s = np.empty(1, np.float32)
-    _check(_get().twq_ref_quant_group_f32(_ptr(v), v.size, _ptr(q), _ptr(s)), "quant_group")
+    fn = _get().twq_ref_quant_group_f32_a8 if a8 else _get().twq_ref_quant_group_f32
+    _check(fn(_ptr(v), v.size, _ptr(q), _ptr(s)), "quant_group")
     return q, float(s[0])
 
 
-def quantize_rows(x_bits):
-    """X (rows x m BF16 bits) -> codes (rows x m int8), scales (rows x m/128 fp32)."""
+def quantize_rows(x_bits, a8=False):
+    """X (rows x m BF16 bits) -> codes (rows x m int8), scales (rows x m/128 fp32);
+    q_max = 7, or 127 for the W4A8 activations (a8)."""
     x = _c(x_bits, np.uint16)
     rows, m = x.shape
     q = np.empty((rows, m), np.int8)
     s = np.empty((rows, m // GROUP), np.float32)
-    _check(_get().twq_ref_quantize_rows(_ptr(x), rows, m, m, _ptr(q), _ptr(s)), "quantize_rows")
+    _check(_get().twq_ref_quantize_rows_q(_ptr(x), rows, m, m, qmax_a8() if a8 else qmax(),
+                                          _ptr(q), _ptr(s)), "quantize_rows")
     return q, s
 
 
@@ -203,9 +214,10 @@ def f32_to_bf16(f: float) -> int:
     return int(_get().twq_ref_f32_to_bf16(f))
 
 
-def layer(x_bits, R, L1, L2, mode=FUSED, rows=None, want=("y",)):
-    """End to end from BF16 inputs: quantize X (rows x m), R, L1, then the layer."""
-    qx, sx = quantize_rows(x_bits)
+def layer(x_bits, R, L1, L2, mode=FUSED, rows=None, want=("y",), a8=False):
+    """End to end from BF16 inputs: quantize X (rows x m), R, L1, then the layer.
+    a8: W4A8, the activations quantized with q_max = 127 (8-bit codes)."""
+    qx, sx = quantize_rows(x_bits, a8=a8)
     qr, sr = quantize_cols(R)
     if L1 is not None and L1.shape[1] > 0:
         ql1, sl1 = quantize_cols(L1)

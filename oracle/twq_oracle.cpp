@@ -35,6 +35,9 @@ namespace {
 constexpr int kGroup = 128;  // §5.1: group size 128
 constexpr int kBits = 4;
 constexpr int kQmax = (1 << (kBits - 1)) - 1;  // Eq. (1): q_max = 2^(k-1) - 1 = 7
+// W4A8 (§5.1, the quantization settings: 4-bit weights, 8-bit activations):
+// the same Eq. (1) with k = 8 for the activations, q_max = 127.
+constexpr int kQmaxA8 = (1 << (8 - 1)) - 1;
 
 float bf16_to_f32(uint16_t h) {
   uint32_t u = static_cast<uint32_t>(h) << 16;
@@ -58,21 +61,21 @@ uint16_t f32_to_bf16(float f) {
 // rounded float division per element. An all-zero group has s = 0 and q = 0
 // (Eq. (1) is 0/0 there).
 void quantize_group(const float* v, int64_t stride, int count, int8_t* q, int64_t qstride,
-                    float* s_out) {
+                    float* s_out, int qmax = kQmax) {
   float a = 0.0f;
   for (int k = 0; k < count; ++k) {
     float m = std::fabs(v[k * stride]);
     if (m > a) a = m;
   }
-  float s = a / static_cast<float>(kQmax);
+  float s = a / static_cast<float>(qmax);
   *s_out = s;
   for (int k = 0; k < count; ++k) {
     int code = 0;
     if (s != 0.0f) {
       float t = v[k * stride] / s;
       float rounded = std::nearbyint(t);  // default rounding mode: half to even
-      if (rounded > kQmax) rounded = kQmax;
-      if (rounded < -kQmax) rounded = -kQmax;
+      if (rounded > qmax) rounded = static_cast<float>(qmax);
+      if (rounded < -qmax) rounded = static_cast<float>(-qmax);
       code = static_cast<int>(rounded);
     }
     q[k * qstride] = static_cast<int8_t>(code);
@@ -94,19 +97,36 @@ int twq_ref_quant_group_f32(const float* v, int count, int8_t* q, float* s) {
   return 0;
 }
 
+int twq_ref_qmax_a8() { return kQmaxA8; }
+
 // Activation codes: X is rows x m BF16 (row stride ldx elements); groups of 128
-// run along m within each row (one scale per token and group).
+// run along m within each row (one scale per token and group). qmax is 7 (W4A4)
+// or 127 (the W4A8 activations).
 // q: rows x m codes (row-major), s: rows x (m/128) scales (row-major).
-int twq_ref_quantize_rows(const uint16_t* x, int64_t rows, int64_t m, int64_t ldx, int8_t* q,
-                          float* s) {
+int twq_ref_quantize_rows_q(const uint16_t* x, int64_t rows, int64_t m, int64_t ldx, int qmax,
+                            int8_t* q, float* s) {
   if (!x || !q || !s || rows < 0 || m <= 0 || m % kGroup || ldx < m) return 1;
+  if (qmax != kQmax && qmax != kQmaxA8) return 1;
   const int64_t G = m / kGroup;
   float buf[kGroup];
   for (int64_t i = 0; i < rows; ++i)
     for (int64_t g = 0; g < G; ++g) {
       for (int k = 0; k < kGroup; ++k) buf[k] = bf16_to_f32(x[i * ldx + g * kGroup + k]);
-      quantize_group(buf, 1, kGroup, q + i * m + g * kGroup, 1, s + i * G + g);
+      quantize_group(buf, 1, kGroup, q + i * m + g * kGroup, 1, s + i * G + g, qmax);
     }
+  return 0;
+}
+
+int twq_ref_quantize_rows(const uint16_t* x, int64_t rows, int64_t m, int64_t ldx, int8_t* q,
+                          float* s) {
+  return twq_ref_quantize_rows_q(x, rows, m, ldx, kQmax, q, s);
+}
+
+// Eq. (1) with q_max = 127 on one group of float inputs (pins on values BF16
+// cannot hold).
+int twq_ref_quant_group_f32_a8(const float* v, int count, int8_t* q, float* s) {
+  if (!v || !q || !s || count <= 0) return 1;
+  quantize_group(v, 1, count, q, 1, s, kQmaxA8);
   return 0;
 }
 

@@ -183,6 +183,42 @@ TWQ_API twq_status twq_fused_linear_x_host(const uint16_t* x_host, int64_t b, co
                                            uint16_t* x_dev, uint16_t* y_dev, uint16_t* y_host,
                                            twq_stream_t stream);
 
+/*
+ * W4A8: 4-bit weights with 8-bit activations, the second quantization setting
+ * of TwinQuant §5.1. The activations use Eq. (1) with k = 8 (q_max = 127), in
+ * groups of 128 along m with one FP32 scale per token and group; the weights
+ * and the rest of the layer are those of twq_fused_linear (same twq_weights).
+ *
+ * twq_quantize_act_a8: x b x m BF16 (row stride ldx, ldx % 8 == 0) ->
+ *   xq8  b x m int8 codes, row-major, element k of a row in byte k;
+ *   sx   b x (m/128) FP32 scales.
+ * Codes and scales are bitwise those of Eq. (1) with correctly rounded float
+ * divisions, round half to even. Errors as twq_quantize_act.
+ */
+TWQ_API twq_status twq_quantize_act_a8(const uint16_t* x, int64_t b, int64_t m, int64_t ldx,
+                                       int8_t* xq8, float* sx, twq_stream_t stream);
+
+/*
+ * The fused W4A8 layer (decode shapes): Y = bf16(Q8(X)Q(R) + bf16(Q8(X)Q(L1)) L2),
+ * each group's int8 x int4 dot product exact in the int32 accumulator (|sum| <=
+ * 128 * 127 * 7), scaled per group in FP32 as in twq_fused_linear.
+ *   xq8, sx  from twq_quantize_act_a8;  w  from twq_pack_weights;  y  b x n BF16.
+ * w->r == 0 gives the residual component alone. Runs the decode kernel, so the
+ * limits are those of twq_fused_linear_x (1 <= b <= 16, m <= 8192, r <= 128);
+ * other shapes return TWQ_ERR_UNSUPPORTED and launch nothing. Launched with
+ * programmatic stream serialization like twq_fused_linear.
+ */
+TWQ_API twq_status twq_fused_linear_a8(const int8_t* xq8, const float* sx, int64_t b,
+                                       const twq_weights* w, uint16_t* y, twq_stream_t stream);
+
+/*
+ * twq_fused_linear_a8 with the 8-bit activation quantizer inside the layer
+ * kernel (one launch, BF16 X in). Bitwise identical to twq_quantize_act_a8
+ * followed by twq_fused_linear_a8. Arguments and limits as twq_fused_linear_x.
+ */
+TWQ_API twq_status twq_fused_linear_x_a8(const uint16_t* x, int64_t ldx, int64_t b,
+                                         const twq_weights* w, uint16_t* y, twq_stream_t stream);
+
 /* Residual component only: Y = bf16(Q(X) Q(R)) (TwinQuant Eq. (2)); ignores l1q/sl1/l2t. */
 TWQ_API twq_status twq_w4a4_only(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
                          uint16_t* y, twq_stream_t stream);

@@ -104,6 +104,17 @@ twq_status twq_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+twq_status twq_quantize_act_a8(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, int8_t* xq8,
+                               float* sx, twq_stream_t stream) {
+  if (b < 0 || m <= 0 || m % 128 || ldx < m) return TWQ_ERR_INVALID_ARG;
+  if (m > (int64_t(1) << 24) || b > (int64_t(1) << 30)) return TWQ_ERR_UNSUPPORTED;
+  if (b == 0) return TWQ_OK;
+  if (!x || !xq8 || !sx) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq8) || !aligned16(sx) || ldx % 8) return TWQ_ERR_MISALIGNED;
+  return from_cuda(twq::launch_quantize_act(x, b, m, ldx, reinterpret_cast<uint8_t*>(xq8), sx,
+                                            reinterpret_cast<cudaStream_t>(stream), true));
+}
+
 twq_status twq_pack_weights(const uint16_t* R, const uint16_t* L1, const uint16_t* L2,
                             const twq_weights* w, twq_stream_t stream) {
   if (!w) return TWQ_ERR_INVALID_ARG;
@@ -146,9 +157,21 @@ twq_status twq_lowrank_only(const uint8_t* xq, const float* sx, int64_t b, const
   return run(twq::kModeLowRank, xq, sx, b, w, y, nullptr, stream);
 }
 
+twq_status twq_fused_linear_a8(const int8_t* xq8, const float* sx, int64_t b, const twq_weights* w,
+                               uint16_t* y, twq_stream_t stream) {
+  const bool lr = w && w->r > 0;
+  const uint8_t* xq = reinterpret_cast<const uint8_t*>(xq8);
+  twq_status s = check_layer(xq, sx, b, w, y, true, lr);
+  if (s != TWQ_OK || b == 0) return s;
+  twq::GemmCall c{lr ? twq::kModeFused : twq::kModeW4A4, xq, sx, b, w, y, nullptr};
+  c.a8 = true;
+  if (!twq::decode_eligible(c)) return TWQ_ERR_UNSUPPORTED;
+  return from_cuda(twq::launch_decode(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 // Validates a twq_fused_linear_x call (b >= 1) and fills the decode launch.
 static twq_status prepare_fused_x(const uint16_t* x, int64_t ldx, int64_t b, const twq_weights* w,
-                                  uint16_t* y, twq::GemmCall* out) {
+                                  uint16_t* y, twq::GemmCall* out, bool a8 = false) {
   if (!x || !y || !w->rq || !w->sr) return TWQ_ERR_INVALID_ARG;
   if (!aligned16(x) || ldx % 8 || !aligned16(y) || !aligned16(w->rq) || !aligned16(w->sr))
     return TWQ_ERR_MISALIGNED;
@@ -160,6 +183,7 @@ static twq_status prepare_fused_x(const uint16_t* x, int64_t ldx, int64_t b, con
   twq::GemmCall c{lr ? twq::kModeFused : twq::kModeW4A4, nullptr, nullptr, b, w, y, nullptr};
   c.x = x;
   c.ldx = ldx;
+  c.a8 = a8;
   if (!twq::decode_eligible(c)) return TWQ_ERR_UNSUPPORTED;
   *out = c;
   return TWQ_OK;
@@ -174,6 +198,18 @@ twq_status twq_fused_linear_x(const uint16_t* x, int64_t ldx, int64_t b, const t
   if (b == 0) return TWQ_OK;
   twq::GemmCall c{};
   if ((s = prepare_fused_x(x, ldx, b, w, y, &c)) != TWQ_OK) return s;
+  return from_cuda(twq::launch_decode(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+twq_status twq_fused_linear_x_a8(const uint16_t* x, int64_t ldx, int64_t b, const twq_weights* w,
+                                 uint16_t* y, twq_stream_t stream) {
+  if (!w) return TWQ_ERR_INVALID_ARG;
+  twq_status s = shape_ok(w->m, w->n, w->r);
+  if (s != TWQ_OK) return s;
+  if (b < 0 || ldx < w->m) return TWQ_ERR_INVALID_ARG;
+  if (b == 0) return TWQ_OK;
+  twq::GemmCall c{};
+  if ((s = prepare_fused_x(x, ldx, b, w, y, &c, true)) != TWQ_OK) return s;
   return from_cuda(twq::launch_decode(c, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -243,11 +279,12 @@ twq_status twq_device_status(int* code) {
 
 int twq_launches_per_call(const char* ep) {
   if (!ep) return -1;
-  if (!strcmp(ep, "twq_quantize_act")) return 1;
+  if (!strcmp(ep, "twq_quantize_act") || !strcmp(ep, "twq_quantize_act_a8")) return 1;
   if (!strcmp(ep, "twq_pack_weights")) return 3;
   if (!strcmp(ep, "twq_fused_linear") || !strcmp(ep, "twq_w4a4_only") ||
       !strcmp(ep, "twq_lowrank_only") || !strcmp(ep, "twq_fused_linear_x") ||
-      !strcmp(ep, "twq_fused_linear_x_host"))
+      !strcmp(ep, "twq_fused_linear_x_host") || !strcmp(ep, "twq_fused_linear_a8") ||
+      !strcmp(ep, "twq_fused_linear_x_a8"))
     return 1;
   if (!strcmp(ep, "twq_unfused_linear") || !strcmp(ep, "twq_unfused_linear_noalloc")) return 4;
   if (!strcmp(ep, "twq_fold_transforms")) return 5;

@@ -178,6 +178,19 @@ __device__ __forceinline__ uint4 pack_codes16(const uint32_t (&nb)[16]) {
   return o;
 }
 
+// 16 int8 codes (q_max = 127) in the same in-chunk order as pack_codes16.
+__device__ __forceinline__ uint4 pack_codes16_a8(const uint32_t (&c)[16]) {
+  uint4 o;
+  o.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+  o.y = c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24);
+  o.z = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+  o.w = c[12] | (c[13] << 8) | (c[14] << 16) | (c[15] << 24);
+  return o;
+}
+
+// kA8: the W4A8 activations (q_max = 127): one int8 code q per byte, the same
+// in-chunk order; else 16*q from a 4-bit code.
+template <bool kA8>
 __device__ __forceinline__ void quantize_slice(const uint8_t* xs, int ng, uint8_t* xu, float* sxs,
                                                uint64_t* xready, int qi, int lane) {
   const int l = lane & 3;
@@ -212,14 +225,15 @@ __device__ __forceinline__ void quantize_slice(const uint8_t* xs, int ng, uint8_
     float a = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 #pragma unroll
     for (int off = 2; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-    const Eq1Scale ks = eq1_scale(a);
+    constexpr int kQmax = kA8 ? 127 : 7;
+    const Eq1Scale ks = eq1_scale<kQmax>(a);
     uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
     if (ks.s != 0.0f) {
       uint32_t nb[16];
-      eq1_nibbles(f[0], ks, nb);
-      o0 = pack_codes16(nb);
-      eq1_nibbles(f[1], ks, nb);
-      o1 = pack_codes16(nb);
+      eq1_codes<kQmax>(f[0], ks, nb);
+      o0 = kA8 ? pack_codes16_a8(nb) : pack_codes16(nb);
+      eq1_codes<kQmax>(f[1], ks, nb);
+      o1 = kA8 ? pack_codes16_a8(nb) : pack_codes16(nb);
     }
     if (pv) {
       *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(t, l)) = o0;
@@ -247,7 +261,8 @@ __device__ __forceinline__ void unit_range(int U, int KS, int k, int& u0, int& u
   u1 = (k + 1) * U / KS;
 }
 
-template <int kMode, int KS, bool kQ>
+// kA8: W4A8, the activation codes are int8 (q_max = 127), one per byte.
+template <int kMode, int KS, bool kQ, bool kA8>
 __global__ void __launch_bounds__(kThreads, 1)
     twq_decode_kernel(const __grid_constant__ CUtensorMap tm_rq,
                       const __grid_constant__ CUtensorMap tm_l1q,
@@ -255,6 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_l2t, const DecodeArgs args) {
   using L = DLayout;
   using T = DTraits<kMode>;
+  // The weight operand holds 16*q (4-bit codes); X holds 16*q (W4A4) or q (W4A8):
+  // an accumulator is 2^8 (2^4) times the group's integer dot product.
+  constexpr float kDq = kA8 ? 0.0625f : 0.00390625f;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int s_abort;
   uint8_t* smem = d_align1024(smem_raw);
@@ -391,8 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(xp + gi * 4096 + 2048, &tm_xq, xfull, (g0 + gi) * 128 + 64, 0);
       }
     } else {
-      mbar_arrive_expect_tx(xfull, ng * 1024);
-      for (int gi = 0; gi < ng; ++gi) tma_load_2d(xp + gi * 1024, &tm_xq, xfull, (g0 + gi) * 64, 0);
+      constexpr int kXBytes = kA8 ? 2048 : 1024;  // one group of 16 tokens: int8 or packed codes
+      mbar_arrive_expect_tx(xfull, ng * kXBytes);
+      for (int gi = 0; gi < ng; ++gi)
+        tma_load_2d(xp + gi * kXBytes, &tm_xq, xfull, (g0 + gi) * (kXBytes / kNT), 0);
     }
   }
   __syncwarp();
@@ -401,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----- X quantize (warps 2-3 and 12-19; 12-19 then go on to their own roles)
     const int qi = (warp < 4 ? warp - 2 : warp - 10) * 32 + lane;
     pdl_wait();
-    if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) quantize_slice(xp, ng, xu, sxs, xready, qi, lane);
+    if (d_wait<false>(xfull, 0, abort_flag, kDSiteX)) quantize_slice<kA8>(xp, ng, xu, sxs, xready, qi, lane);
   }
   if (warp == 0) {
     // ------------------------------------ residual MMA issuer (lane 0 of warp 0)
@@ -492,9 +512,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int gi = e / (kNT * 8);
           const int row = (e / 8) % kNT;
           const int c = e & 7;
-          const uint2 w = *reinterpret_cast<const uint2*>(xp + gi * 1024 + row * 64 + c * 8);
           uint32_t o[4];
-          unpack8(w.x, w.y, o);
+          if constexpr (kA8) {  // 16 int8 codes in element order -> the MMA's in-chunk order
+            const uint4 w = *reinterpret_cast<const uint4*>(xp + gi * 2048 + row * 128 + c * 16);
+            o[0] = __byte_perm(w.x, w.y, 0x6420);  // elements 0, 2, 4, 6
+            o[1] = __byte_perm(w.x, w.y, 0x7531);  // 1, 3, 5, 7
+            o[2] = __byte_perm(w.z, w.w, 0x6420);  // 8, 10, 12, 14
+            o[3] = __byte_perm(w.z, w.w, 0x7531);  // 9, 11, 13, 15
+          } else {
+            const uint2 w = *reinterpret_cast<const uint2*>(xp + gi * 1024 + row * 64 + c * 8);
+            unpack8(w.x, w.y, o);
+          }
           *reinterpret_cast<uint4*>(xu + gi * 2048 + d_sw128(row, c)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
 #pragma unroll
@@ -586,8 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t rbar = map_peer(smem_u32(h_ready), owner);
 #pragma unroll
         for (int t = 0; t < kNT; t += 4)
-          st_async_peer_v4(dst + t * 4, acc[t] * 0.00390625f, acc[t + 1] * 0.00390625f,
-                           acc[t + 2] * 0.00390625f, acc[t + 3] * 0.00390625f, rbar);
+          st_async_peer_v4(dst + t * 4, acc[t] * kDq, acc[t + 1] * kDq, acc[t + 2] * kDq,
+                           acc[t + 3] * kDq, rbar);
       }
       // An owner waits until every peer's bytes have landed (so none is still writing
       // into it when it exits); the wait ignores the abort flag for the same reason.
@@ -641,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     float part[kNT];
 #pragma unroll
-    for (int t = 0; t < kNT; ++t) part[t] = acc[t] * 0.00390625f;
+    for (int t = 0; t < kNT; ++t) part[t] = acc[t] * kDq;
     if (T::lr && my_units > 0 && ok) {
       if ((ok = d_wait<false>(lr_full, 0, abort_flag, kDSiteLr))) {
         tc_fence_after();
@@ -728,7 +756,7 @@ bool d_encode(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int kMode, int KS, bool kQ>
+template <int kMode, int KS, bool kQ, bool kA8>
 cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
   const twq_weights* w = c.w;
   DecodeArgs a{};
@@ -745,8 +773,10 @@ cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
   const uint64_t kb = static_cast<uint64_t>(a.m / 2);
   bool ok = kQ ? d_encode(&m_xq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.x, a.m, c.b,
                           static_cast<uint64_t>(c.ldx) * 2, 64, kNT, CU_TENSOR_MAP_SWIZZLE_NONE)
-                : d_encode(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, kb, c.b, kb, 64, kNT,
-                           CU_TENSOR_MAP_SWIZZLE_NONE);
+           : kA8 ? d_encode(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, a.m, c.b, a.m, 128, kNT,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)
+                 : d_encode(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, kb, c.b, kb, 64, kNT,
+                            CU_TENSOR_MAP_SWIZZLE_NONE);
   if (DTraits<kMode>::res)
     ok = ok && d_encode(&m_rq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->rq, kb, a.n, kb, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_64B);
@@ -757,7 +787,7 @@ cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
     ok = ok && d_encode(&m_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2t, a.r, a.n,
                         static_cast<uint64_t>(a.r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
-  auto kern = twq_decode_kernel<kMode, KS, kQ>;
+  auto kern = twq_decode_kernel<kMode, KS, kQ, kA8>;
   // The shared-memory opt-in is a driver call: once per instantiation and device.
   static std::atomic<uint64_t> smem_set{0};
   int dev = 0;
@@ -796,6 +826,7 @@ cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
 bool decode_eligible(const GemmCall& c) {
   const twq_weights* w = c.w;
   if (c.mode != kModeFused && c.mode != kModeW4A4 && c.mode != kModeLowRank) return false;
+  if (c.a8 && c.mode == kModeLowRank) return false;
   if (c.b < 1 || c.b > kNT) return false;
   if (c.mode != kModeW4A4 && (w->r <= 0 || w->r > 128)) return false;
   const int64_t G = w->m / 128;
@@ -806,14 +837,23 @@ cudaError_t launch_decode(const GemmCall& c, cudaStream_t st) {
   const int64_t G = c.w->m / 128;
   const bool ks8 = G > 4 * kMaxGroups;
   const bool q = c.x != nullptr;
-#define TWQ_DECODE_CASE(MODE)                                                         \
-  if (q) return ks8 ? launch_decode_mode<MODE, 8, true>(c, st)                       \
-                    : launch_decode_mode<MODE, 4, true>(c, st);                      \
-  return ks8 ? launch_decode_mode<MODE, 8, false>(c, st) : launch_decode_mode<MODE, 4, false>(c, st);
+#define TWQ_DECODE_CASE(MODE, A8)                                                          \
+  if (q) return ks8 ? launch_decode_mode<MODE, 8, true, A8>(c, st)                        \
+                    : launch_decode_mode<MODE, 4, true, A8>(c, st);                       \
+  return ks8 ? launch_decode_mode<MODE, 8, false, A8>(c, st)                              \
+             : launch_decode_mode<MODE, 4, false, A8>(c, st);
+  if (c.a8) {  // W4A8: the full layer and the residual alone
+    switch (c.mode) {
+      case kModeFused: { TWQ_DECODE_CASE(kModeFused, true) }
+      case kModeW4A4: { TWQ_DECODE_CASE(kModeW4A4, true) }
+      default:
+        return cudaErrorInvalidValue;
+    }
+  }
   switch (c.mode) {
-    case kModeFused: { TWQ_DECODE_CASE(kModeFused) }
-    case kModeW4A4: { TWQ_DECODE_CASE(kModeW4A4) }
-    case kModeLowRank: { TWQ_DECODE_CASE(kModeLowRank) }
+    case kModeFused: { TWQ_DECODE_CASE(kModeFused, false) }
+    case kModeW4A4: { TWQ_DECODE_CASE(kModeW4A4, false) }
+    case kModeLowRank: { TWQ_DECODE_CASE(kModeLowRank, false) }
     default:
       return cudaErrorInvalidValue;
   }

@@ -28,12 +28,14 @@ struct GemmCall {
   const uint16_t* h_global; // kModeS2F32 only: bf16 H, b x r
   const uint16_t* x = nullptr;  // decode kernel only: BF16 X, quantized in the kernel
   int64_t ldx = 0;
+  bool a8 = false;  // W4A8 (decode kernel only): xq holds int8 codes (q_max = 127), b x m
 };
 
 // Host-side launchers; all return cudaSuccess or the launch error.
 cudaError_t launch_gemm(const GemmCall& call, cudaStream_t stream, int* launches);
+// a8: int8 codes with q_max = 127 (b x m bytes), else packed nibbles (b x m/2 bytes).
 cudaError_t launch_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
-                                float* sx, cudaStream_t stream);
+                                float* sx, cudaStream_t stream, bool a8 = false);
 cudaError_t launch_pack_cols(const uint16_t* w, int64_t m, int64_t cols, uint8_t* q, float* s,
                              cudaStream_t stream);
 cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out,

@@ -16,6 +16,9 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as
 
 // One half-warp per (token, group): lane l of the half covers elements
 // [8l, 8l + 8) of the group; a warp covers two consecutive groups of one row.
+// kA8: q_max = 127, one int8 code per element (W4A8 activations); else q_max = 7,
+// two nibbles per byte.
+template <bool kA8>
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x,
                                                            int64_t b, int m, int64_t ldx,
                                                            uint8_t* __restrict__ xq,
@@ -48,17 +51,22 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
   for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(f[k]));
 #pragma unroll
   for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-  const Eq1Scale ks = eq1_scale(a);
+  constexpr int kQmax = kA8 ? 127 : 7;
+  const Eq1Scale ks = eq1_scale<kQmax>(a);
   const float s = ks.s;
-  uint32_t word = 0;
-  if (s != 0.0f) {
-    uint32_t nib[8];
-    eq1_nibbles(f, ks, nib);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) word |= nib[k] << (4 * k);
-  }
+  uint32_t code[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (s != 0.0f) eq1_codes<kQmax>(f, ks, code);
   if (valid) {
-    *reinterpret_cast<uint32_t*>(xq + row * (m / 2) + g * 64 + l * 4) = word;
+    if constexpr (kA8) {  // element 8l + k in byte k
+      const uint2 v = make_uint2(code[0] | (code[1] << 8) | (code[2] << 16) | (code[3] << 24),
+                                 code[4] | (code[5] << 8) | (code[6] << 16) | (code[7] << 24));
+      *reinterpret_cast<uint2*>(xq + row * m + g * 128 + l * 8) = v;
+    } else {  // element 8l + k in nibble k (element 2p in the low nibble of byte p)
+      uint32_t word = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) word |= code[k] << (4 * k);
+      *reinterpret_cast<uint32_t*>(xq + row * (m / 2) + g * 64 + l * 4) = word;
+    }
     if (l == 0) sx[row * G + g] = s;
   }
 }
@@ -131,12 +139,16 @@ __global__ void add_cast_kernel(const float4* __restrict__ a, const float4* __re
 }  // namespace
 
 cudaError_t launch_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
-                                float* sx, cudaStream_t st) {
+                                float* sx, cudaStream_t st, bool a8) {
   const int G = static_cast<int>(m / 128);
   const int64_t warps = b * ((G + 1) / 2);
   const int64_t blocks = (warps + 7) / 8;
-  quantize_act_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(x, b, static_cast<int>(m),
-                                                                     ldx, xq, sx);
+  if (a8)
+    quantize_act_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        x, b, static_cast<int>(m), ldx, xq, sx);
+  else
+    quantize_act_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        x, b, static_cast<int>(m), ldx, xq, sx);
   return cudaGetLastError();
 }
 

@@ -28,7 +28,8 @@ EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_siz
            "twq_lowrank_only", "twq_unfused_workspace_bytes", "twq_unfused_linear",
            "twq_device_status", "twq_launches_per_call", "twq_unfused_linear_noalloc",
            "twq_fused_linear_x", "twq_fold_workspace_bytes", "twq_fold_transforms",
-           "twq_fused_linear_x_host")
+           "twq_fused_linear_x_host", "twq_quantize_act_a8", "twq_fused_linear_a8",
+           "twq_fused_linear_x_a8")
 
 
 class TwqError(RuntimeError):
@@ -73,6 +74,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twq_unfused_linear_noalloc": ([P, P, I, P, P, P], ctypes.c_int),
         "twq_fused_linear_x": ([P, I, I, P, P, P], ctypes.c_int),
         "twq_fused_linear_x_host": ([P, I, P, P, P, P, P], ctypes.c_int),
+        "twq_quantize_act_a8": ([P, I, I, I, P, P, P], ctypes.c_int),
+        "twq_fused_linear_a8": ([P, P, I, P, P, P], ctypes.c_int),
+        "twq_fused_linear_x_a8": ([P, I, I, P, P, P], ctypes.c_int),
         "twq_fold_workspace_bytes": ([I, I, I], S),
         "twq_fold_transforms": ([P, P, P, P, P, I, I, I, P, P, P, P, S, P], ctypes.c_int),
     }
@@ -203,9 +207,36 @@ def fused_linear(xq, sx, w: Weights, y=None, stream=None):
     return _layer("twq_fused_linear", xq, sx, w, y, stream)
 
 
-def fused_linear_x(x: torch.Tensor, w: Weights, y=None, stream=None):
+def quantize_act_a8(x: torch.Tensor, xq8: torch.Tensor | None = None,
+                    sx: torch.Tensor | None = None, stream=None):
+    """W4A8 activations: BF16 X (b x m) -> int8 codes (b x m, q_max = 127) and scales
+    (b x m/128 fp32)."""
+    b, m = x.shape
+    if xq8 is None:
+        xq8 = torch.empty((b, m), dtype=torch.int8, device=x.device)
+    if sx is None:
+        sx = torch.empty((b, max(m // 128, 1)), dtype=torch.float32, device=x.device)
+    _check(load().twq_quantize_act_a8(_dev(x, "x", torch.bfloat16), b, m, m,
+                                      _dev(xq8, "xq8", torch.int8), _dev(sx, "sx", torch.float32),
+                                      _stream(stream)), "twq_quantize_act_a8")
+    return xq8, sx
+
+
+def fused_linear_a8(xq8, sx, w: Weights, y=None, stream=None):
+    """The fused W4A8 layer on codes from quantize_act_a8 (decode batches, b <= 16)."""
+    b = xq8.shape[0]
+    if y is None:
+        y = torch.empty((b, w.n), dtype=torch.bfloat16, device=xq8.device)
+    cw = w.c_struct()
+    _check(load().twq_fused_linear_a8(_dev(xq8, "xq8", torch.int8), _dev(sx, "sx", torch.float32),
+                                      b, ctypes.byref(cw), _dev(y, "y", torch.bfloat16),
+                                      _stream(stream)), "twq_fused_linear_a8")
+    return y
+
+
+def fused_linear_x(x: torch.Tensor, w: Weights, y=None, stream=None, a8: bool = False):
     """BF16 X (b x m, rows may be strided) -> Y in one launch, quantizing X inside
-    the layer kernel (decode batches, b <= 16)."""
+    the layer kernel (decode batches, b <= 16). a8: W4A8 (8-bit activation codes)."""
     if not isinstance(x, torch.Tensor) or x.dim() != 2:
         raise TypeError("x must be a 2-D torch tensor")
     if not x.is_cuda:
@@ -219,9 +250,9 @@ def fused_linear_x(x: torch.Tensor, w: Weights, y=None, stream=None):
     if y is None:
         y = torch.empty((b, w.n), dtype=torch.bfloat16, device=x.device)
     cw = w.c_struct()
-    _check(load().twq_fused_linear_x(x.data_ptr(), ldx, b, ctypes.byref(cw),
-                                     _dev(y, "y", torch.bfloat16), _stream(stream)),
-           "twq_fused_linear_x")
+    fn = "twq_fused_linear_x_a8" if a8 else "twq_fused_linear_x"
+    _check(getattr(load(), fn)(x.data_ptr(), ldx, b, ctypes.byref(cw),
+                               _dev(y, "y", torch.bfloat16), _stream(stream)), fn)
     return y
 
 

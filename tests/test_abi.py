@@ -141,6 +141,31 @@ def test_fused_linear_x_host_validation(lib):
     assert f(A, 4, ctypes.byref(_w(r=144)), A, A, A, None) == 2
 
 
+def test_w4a8_validation(lib):
+    # every rejection happens before anything is launched
+    q = lib.twq_quantize_act_a8
+    assert q(None, 4, 512, 512, A, A, None) == 1
+    assert q(A, 4, 500, 512, A, A, None) == 1            # m % 128
+    assert q(A, 4, 512, 256, A, A, None) == 1            # ldx < m
+    assert q(A, 4, 512, 516, A, A, None) == 3            # row stride breaks 16 bytes
+    assert q(A, 4, 512, 512, A + 8, A, None) == 3
+    assert q(None, 0, 512, 512, None, None, None) == 0   # b == 0: nothing to do
+    f = lib.twq_fused_linear_a8
+    w = _w()
+    assert f(None, A, 4, ctypes.byref(w), A, None) == 1
+    assert f(A, A, 4, None, A, None) == 1
+    assert f(A + 4, A, 4, ctypes.byref(w), A, None) == 3
+    assert f(A, A, 17, ctypes.byref(w), A, None) == 2     # prefill batches: not on this path
+    assert f(A, A, 4, ctypes.byref(_w(r=144)), A, None) == 2
+    assert f(A, A, 0, ctypes.byref(w), None, None) == 0
+    fx = lib.twq_fused_linear_x_a8
+    assert fx(None, 512, 4, ctypes.byref(w), A, None) == 1
+    assert fx(A, 256, 4, ctypes.byref(w), A, None) == 1
+    assert fx(A, 516, 4, ctypes.byref(w), A, None) == 3
+    assert fx(A, 512, 17, ctypes.byref(w), A, None) == 2
+    assert fx(A, 512, 0, ctypes.byref(w), None, None) == 0
+
+
 def test_fold_validation(lib):
     f = lib.twq_fold_transforms
     ws = lib.twq_fold_workspace_bytes(256, 128, 32)
@@ -184,6 +209,8 @@ def test_launch_accounting(lib):
     assert twq.launches_per_call("twq_unfused_linear_noalloc") == 4
     assert twq.launches_per_call("twq_fused_linear_x") == 1
     assert twq.launches_per_call("twq_fused_linear_x_host") == 1
+    for ep in ("twq_quantize_act_a8", "twq_fused_linear_a8", "twq_fused_linear_x_a8"):
+        assert twq.launches_per_call(ep) == 1
     assert twq.launches_per_call("twq_fold_transforms") == 5
     assert twq.launches_per_call("nope") == -1
 

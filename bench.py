@@ -276,6 +276,12 @@ class Problem:
         c = i % self.copies
         twq.fused_linear_x(self.x[c], self.weights[c], self.y[c])
 
+    def step_x_a8(self, i):
+        """W4A8 (8-bit activation codes), one launch: a comparison, not the metric's step."""
+        from rank_residual_w4a4_b200 import twq
+        c = i % self.copies
+        twq.fused_linear_x(self.x[c], self.weights[c], self.y[c], a8=True)
+
     def step_two_call(self, i):
         from rank_residual_w4a4_b200 import twq
         c = i % self.copies
@@ -390,6 +396,7 @@ def run_gpu(args):
     one = prob.one_launch
     t_fused = kernel_only_time(prob, prob.step_x if one else fused_only, K)
     t_two = time_graph(capture(prob.step_two_call, K), world, device) / K if one else None
+    t_a8 = time_graph(capture(prob.step_x_a8, K), world, device) / K if one else None
     st = twq.device_status()
     if st != 0:
         raise RuntimeError("device wait timed out at site %d" % st)
@@ -435,6 +442,9 @@ def run_gpu(args):
     if one:
         line["two_call_step_us"] = round(t_two * 1e6, 3)
         line["two_call_step"] = "twq_quantize_act + twq_fused_linear, same graph timing"
+        line["w4a8_step_us"] = round(t_a8 * 1e6, 3)
+        line["w4a8_step"] = ("twq_fused_linear_x_a8: the same layer with 8-bit activation codes "
+                             "(W4A8), same graph timing")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(name, seconds=args.cpu_seconds)
     if rank == 0 and world == 1 and not args.no_sweep:
@@ -541,6 +551,7 @@ def sweep(args, device, peaks):
         t_u = kernel_only_time(prob, unf, steps, reps=3)
         t_q = kernel_only_time(prob, quant, steps, reps=3)
         t_x = kernel_only_time(prob, prob.step_x, steps, reps=3) if prob.one_launch else None
+        t_a8 = kernel_only_time(prob, prob.step_x_a8, steps, reps=3) if prob.one_launch else None
         ops = int8_ops(b, wl.m, wl.n, wl.r) + bf16_flops(b, wl.n, wl.r)
         res.update({
             "fused_us": round(t_f * 1e6, 2), "w4a4_only_us": round(t_w * 1e6, 2),
@@ -552,6 +563,7 @@ def sweep(args, device, peaks):
         })
         if t_x is not None:
             res["fused_x_us"] = round(t_x * 1e6, 2)
+            res["fused_x_a8_us"] = round(t_a8 * 1e6, 2)
             res["tokens_per_s"] = round(b / t_x, 1)
             res["roofline_x"] = roofline_entry(name, t_x, peaks, profiled_traffic(name + "_x"),
                                                bf16_x=True)

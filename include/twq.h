@@ -199,14 +199,14 @@ TWQ_API twq_status twq_quantize_act_a8(const uint16_t* x, int64_t b, int64_t m, 
                                        int8_t* xq8, float* sx, twq_stream_t stream);
 
 /*
- * The fused W4A8 layer (decode shapes): Y = bf16(Q8(X)Q(R) + bf16(Q8(X)Q(L1)) L2),
- * each group's int8 x int4 dot product exact in the int32 accumulator (|sum| <=
- * 128 * 127 * 7), scaled per group in FP32 as in twq_fused_linear.
+ * The fused W4A8 layer: Y = bf16(Q8(X)Q(R) + bf16(Q8(X)Q(L1)) L2), each group's
+ * int8 x int4 dot product exact in the int32 accumulator (|sum| <= 128 * 127 * 7),
+ * scaled per group in FP32 as in twq_fused_linear.
  *   xq8, sx  from twq_quantize_act_a8;  w  from twq_pack_weights;  y  b x n BF16.
- * w->r == 0 gives the residual component alone. Runs the decode kernel, so the
- * limits are those of twq_fused_linear_x (1 <= b <= 16, m <= 8192, r <= 128);
- * other shapes return TWQ_ERR_UNSUPPORTED and launch nothing. Launched with
- * programmatic stream serialization like twq_fused_linear.
+ * w->r == 0 gives the residual component alone. Shapes and errors as
+ * twq_fused_linear: decode batches (b <= 16, r <= 128, m <= 8192) run the
+ * split-K decode kernel (with programmatic stream serialization), larger ones the
+ * tensor-core GEMM kernel, whose MMAs read the int8 X tile where TMA stored it.
  */
 TWQ_API twq_status twq_fused_linear_a8(const int8_t* xq8, const float* sx, int64_t b,
                                        const twq_weights* w, uint16_t* y, twq_stream_t stream);

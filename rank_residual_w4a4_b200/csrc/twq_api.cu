@@ -165,8 +165,9 @@ twq_status twq_fused_linear_a8(const int8_t* xq8, const float* sx, int64_t b, co
   if (s != TWQ_OK || b == 0) return s;
   twq::GemmCall c{lr ? twq::kModeFused : twq::kModeW4A4, xq, sx, b, w, y, nullptr};
   c.a8 = true;
-  if (!twq::decode_eligible(c)) return TWQ_ERR_UNSUPPORTED;
-  return from_cuda(twq::launch_decode(c, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (twq::decode_eligible(c)) return from_cuda(twq::launch_decode(c, st));
+  return from_cuda(twq::launch_gemm(c, st, nullptr));
 }
 
 // Validates a twq_fused_linear_x call (b >= 1) and fills the decode launch.

@@ -59,9 +59,13 @@ struct ModeTraits {
   static constexpr bool out_h = kMode == kModeHOnly;
 };
 
-template <int BN>
+// kA8 (W4A8): the X tile is 128 rows x 128 int8 codes, TMA-loaded with the 128-byte
+// swizzle straight into the packed slot, where the MMA reads it (no unpack); three
+// stages of 24 KB instead of four of 16 KB keep the budget.
+template <int BN, bool kA8 = false>
 struct SmemLayout {
-  static constexpr int kSlotA = 8192;  // 128 rows x 64 packed bytes
+  static constexpr int kStages = kA8 ? 3 : kPackedStages;
+  static constexpr int kSlotA = kA8 ? 16384 : 8192;  // 128 rows x 128 int8, or x 64 packed bytes
   static constexpr int kSlot = (kSlotA + BN * 64) > BN * 128 ? (kSlotA + BN * 64) : BN * 128;
   static constexpr int kUA = 16384;   // 128 rows x 128 int8
   static constexpr int kUB = BN * 128;
@@ -69,17 +73,18 @@ struct SmemLayout {
   static constexpr int kHb = kBM * kMaxRank * 2;  // up to 4 K-chunks of 128 x 64 BF16
   static constexpr int kScaleSlot = BN * 4;
   static constexpr int kOffSlots = 0;
-  static constexpr int kOffU = kOffSlots + kPackedStages * kSlot;
+  static constexpr int kOffU = kOffSlots + kStages * kSlot;
   static constexpr int kOffHb = kOffU + kUnpackedStages * kUStage;
   static constexpr int kOffScale = kOffHb + kHb;
   static constexpr int kOffBar = kOffScale + kScaleSlots * kScaleSlot;
   static constexpr int kNumBars =
-      2 * kPackedStages + 2 * kUnpackedStages + 2 * kAccBufs + 2 * kScaleSlots + 4;
+      2 * kStages + 2 * kUnpackedStages + 2 * kAccBufs + 2 * kScaleSlots + 4;
   static constexpr int kBytes = kOffBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
   static constexpr int kTmemCols = kAccBufs * BN;  // accumulator buffers
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
   static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of 2");
+  static_assert(!kA8 || kSlot % 1024 == 0, "a 128-byte-swizzle TMA tile starts on 1 KB");
 };
 
 struct GemmArgs {
@@ -195,6 +200,10 @@ __device__ __forceinline__ UnpackPlan unpack_plan(int tid) {
 
 // Unpacks the first `rows` rows (<= 128) of a tile with the thread's plan; all
 // loads are issued before any store so the shared-memory latencies overlap.
+// kNatural: element order within each 16-byte chunk (to pair with int8 X codes
+// loaded as they are, W4A8), two byte permutes per 8 output bytes; else even
+// elements first, the order both 4-bit operands share.
+template <bool kNatural = false>
 __device__ __forceinline__ void unpack_tile(const uint8_t* src, uint8_t* dst, int rows,
                                             const UnpackPlan& p) {
   uint4 w[3];
@@ -205,14 +214,21 @@ __device__ __forceinline__ void unpack_tile(const uint8_t* src, uint8_t* dst, in
   for (int i = 0; i < 3; ++i) {
     if (p.row[i] < rows) {
       uint4 o0, o1;
-      o0.x = (w[i].x << 4) & 0xF0F0F0F0u;
-      o0.y = w[i].x & 0xF0F0F0F0u;
+      o0.x = (w[i].x << 4) & 0xF0F0F0F0u;  // 16 x elements 0, 2, 4, 6 of the word
+      o0.y = w[i].x & 0xF0F0F0F0u;         // 16 x elements 1, 3, 5, 7
       o0.z = (w[i].y << 4) & 0xF0F0F0F0u;
       o0.w = w[i].y & 0xF0F0F0F0u;
       o1.x = (w[i].z << 4) & 0xF0F0F0F0u;
       o1.y = w[i].z & 0xF0F0F0F0u;
       o1.z = (w[i].w << 4) & 0xF0F0F0F0u;
       o1.w = w[i].w & 0xF0F0F0F0u;
+      if constexpr (kNatural) {
+        const uint4 e0 = o0, e1 = o1;
+        o0 = make_uint4(__byte_perm(e0.x, e0.y, 0x5140), __byte_perm(e0.x, e0.y, 0x7362),
+                        __byte_perm(e0.z, e0.w, 0x5140), __byte_perm(e0.z, e0.w, 0x7362));
+        o1 = make_uint4(__byte_perm(e1.x, e1.y, 0x5140), __byte_perm(e1.x, e1.y, 0x7362),
+                        __byte_perm(e1.z, e1.w, 0x5140), __byte_perm(e1.z, e1.w, 0x7362));
+      }
       *reinterpret_cast<uint4*>(dst + p.dst0[i]) = o0;
       *reinterpret_cast<uint4*>(dst + p.dst1[i]) = o1;
     }
@@ -280,15 +296,20 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, int t, int t_be
 // kPair: a cluster of two CTAs works on the two column tiles of one pair at a
 // time; CTA k computes H columns [k r/2, (k+1) r/2) of the row block and stores
 // its BF16 slice into both CTAs' H operand tiles, so H is computed once per pair.
-template <int kMode, int BN, bool kPair>
+// kA8: W4A8, X as int8 codes (q_max = 127) read by the MMA where TMA put them.
+template <int kMode, int BN, bool kPair, bool kA8>
 __global__ void __launch_bounds__(kThreads, 1)
     twq_gemm_kernel(const __grid_constant__ CUtensorMap tm_xq,
                     const __grid_constant__ CUtensorMap tm_rq,
                     const __grid_constant__ CUtensorMap tm_l1q,
                     const __grid_constant__ CUtensorMap tm_l2t,
                     const __grid_constant__ CUtensorMap tm_h, const GemmArgs args) {
-  using L = SmemLayout<BN>;
+  using L = SmemLayout<BN, kA8>;
   using T = ModeTraits<kMode>;
+  // The weight operand holds 16*q (4-bit codes); X holds 16*q (W4A4) or q (W4A8):
+  // an accumulator is 2^8 (2^4) times the group's integer dot product.
+  constexpr float kDq = kA8 ? 0.0625f : 0.00390625f;
+  constexpr int kStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int s_abort;
   uint8_t* smem = align1024(smem_raw);
@@ -298,8 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* scl = reinterpret_cast<float*>(smem + L::kOffScale);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* full = bars;
-  uint64_t* empty = full + kPackedStages;
-  uint64_t* ufull = empty + kPackedStages;
+  uint64_t* empty = full + kStages;
+  uint64_t* ufull = empty + kStages;
   uint64_t* uempty = ufull + kUnpackedStages;
   uint64_t* acc_full = uempty + kUnpackedStages;
   uint64_t* acc_empty = acc_full + kAccBufs;
@@ -324,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int KC = args.r_pad / 64;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPackedStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 6);
+      mbar_init(&empty[i], kA8 ? 7 : 6);  // the unpack warps (+ the MMA, which reads X there)
     }
     for (int i = 0; i < kUnpackedStages; ++i) {
       mbar_init(&ufull[i], 6);
@@ -389,8 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       Ring s, q;
       uint32_t hb_phase = 0;
       bool hb_pend = false;
-      bool pend[kPackedStages] = {};
-      uint32_t pend_phase[kPackedStages];
+      bool pend[kStages] = {};
+      uint32_t pend_phase[kStages];
       bool spend[kScaleSlots] = {};
       uint32_t spend_phase[kScaleSlots];
       bool ok = true;
@@ -406,11 +427,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
               uint8_t* slot = slots + s.idx * L::kSlot;
               mbar_arrive_expect_tx(&full[s.idx], L::kSlotA + args.h_box * 64);
-              tma_load_2d(slot, &tm_xq, &full[s.idx], g * 64, row0);
+              tma_load_2d(slot, &tm_xq, &full[s.idx], g * (kA8 ? 128 : 64), row0);
               tma_load_2d(slot + L::kSlotA, &tm_l1q, &full[s.idx], g * 64, h_row0(hc));
               pend[s.idx] = true;
               pend_phase[s.idx] = s.phase;
-              s.next(kPackedStages);
+              s.next(kStages);
               if (!(ok = wait_fast(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
                                   kSiteProducerScaleEmpty)))
                 break;
@@ -429,11 +450,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             uint8_t* slot = slots + s.idx * L::kSlot;
             mbar_arrive_expect_tx(&full[s.idx], L::kSlotA + BN * 64);
-            tma_load_2d(slot, &tm_xq, &full[s.idx], g * 64, row0);
+            tma_load_2d(slot, &tm_xq, &full[s.idx], g * (kA8 ? 128 : 64), row0);
             tma_load_2d(slot + L::kSlotA, &tm_rq, &full[s.idx], g * 64, n0);
             pend[s.idx] = true;
             pend_phase[s.idx] = s.phase;
-            s.next(kPackedStages);
+            s.next(kStages);
             if (!(ok = wait_fast(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
                                 kSiteProducerScaleEmpty)))
               break;
@@ -461,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(slots + s.idx * L::kSlot, &tm_l2t, &full[s.idx], kc * 64, n0);
             pend[s.idx] = true;
             pend_phase[s.idx] = s.phase;
-            s.next(kPackedStages);
+            s.next(kStages);
           }
         }
       }
@@ -469,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Aborting: let the copies already issued land before the CTA exits.
         int dummy = 0;
         volatile int* never = &dummy;
-        for (int i = 0; i < kPackedStages; ++i)
+        for (int i = 0; i < kStages; ++i)
           if (pend[i]) wait_fast(&full[i], pend_phase[i], never, kSiteFinal);
         for (int i = 0; i < kScaleSlots; ++i)
           if (spend[i]) wait_fast(&sc_full[i], spend_phase[i], never, kSiteFinal);
@@ -479,11 +500,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      Ring u, a;
+      Ring u, a, s;  // s: the packed slot of each step (W4A8: X is read there)
       uint32_t hb_phase = 0;
       bool ok = true;
       const uint32_t ua0 = smem_u32(ustg);
       const uint32_t hb0 = smem_u32(hb);
+      const uint32_t slot0 = smem_u32(slots);
+      // W4A8: the step's packed slot is released by the unpack warps and by this commit
+      auto release_slot = [&]() {
+        if constexpr (kA8) mma_commit(&empty[s.idx]);
+        s.next(kStages);
+      };
       for (int t = t_begin; t < t_end && ok; ++t) {
         const TileInfo ti = tile_info(args, t, t_begin, T::h, kPairStride, prank);
         if (ti.need_h) {
@@ -496,12 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
               tc_fence_after();
               const uint32_t d = tmem_base + a.idx * BN;
-              const uint64_t da = smem_desc_sw128(ua0 + u.idx * L::kUStage);
+              const uint64_t da = kA8 ? smem_desc_sw128(slot0 + s.idx * L::kSlot)
+                                      : smem_desc_sw128(ua0 + u.idx * L::kUStage);
               const uint64_t db = smem_desc_sw128(ua0 + u.idx * L::kUStage + L::kUA);
 #pragma unroll
               for (int k = 0; k < 4; ++k) mma_i8(d, da + 2 * k, db + 2 * k, idesc, k > 0);
               mma_commit(&uempty[u.idx]);
               mma_commit(&acc_full[a.idx]);
+              release_slot();
               u.next(kUnpackedStages);
               a.next(kAccBufs);
             }
@@ -515,12 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             tc_fence_after();
             const uint32_t d = tmem_base + a.idx * BN;
-            const uint64_t da = smem_desc_sw128(ua0 + u.idx * L::kUStage);
+            const uint64_t da = kA8 ? smem_desc_sw128(slot0 + s.idx * L::kSlot)
+                                    : smem_desc_sw128(ua0 + u.idx * L::kUStage);
             const uint64_t db = smem_desc_sw128(ua0 + u.idx * L::kUStage + L::kUA);
 #pragma unroll
             for (int k = 0; k < 4; ++k) mma_i8(d, da + 2 * k, db + 2 * k, idesc, k > 0);
             mma_commit(&uempty[u.idx]);
             mma_commit(&acc_full[a.idx]);
+            release_slot();
             u.next(kUnpackedStages);
             a.next(kAccBufs);
           }
@@ -549,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 4; ++k)
               mma_bf16(d, da + 2 * k, db + 2 * k, idesc, (kc | k) != 0);
             mma_commit(&uempty[u.idx]);
+            release_slot();
             u.next(kUnpackedStages);
           }
           if (!ok) break;
@@ -585,8 +617,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int hc = step / G;
             brows = h_cols(hc);
           }
-          unpack_tile(src, dst, kBM, plan);
-          unpack_tile(src + L::kSlotA, dst + L::kUA, brows, plan);
+          if constexpr (!kA8) unpack_tile(src, dst, kBM, plan);  // W4A8: the MMA reads X in place
+          unpack_tile<kA8>(src + L::kSlotA, dst + L::kUA, brows, plan);
         } else {
           copy_smem(src, dst + L::kUA, BN * 128, tid, 192);
         }
@@ -596,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&ufull[u.idx]);
           mbar_arrive(&empty[s.idx]);
         }
-        s.next(kPackedStages);
+        s.next(kStages);
         u.next(kUnpackedStages);
       }
     }
@@ -662,10 +694,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 64; j += 8) {
             if (j < ncols) {
               uint4 o;
-              o.x = pack_bf16x2(acc[j + 0] * 0.00390625f, acc[j + 1] * 0.00390625f);
-              o.y = pack_bf16x2(acc[j + 2] * 0.00390625f, acc[j + 3] * 0.00390625f);
-              o.z = pack_bf16x2(acc[j + 4] * 0.00390625f, acc[j + 5] * 0.00390625f);
-              o.w = pack_bf16x2(acc[j + 6] * 0.00390625f, acc[j + 7] * 0.00390625f);
+              o.x = pack_bf16x2(acc[j + 0] * kDq, acc[j + 1] * kDq);
+              o.y = pack_bf16x2(acc[j + 2] * kDq, acc[j + 3] * kDq);
+              o.z = pack_bf16x2(acc[j + 4] * kDq, acc[j + 5] * kDq);
+              o.w = pack_bf16x2(acc[j + 6] * kDq, acc[j + 7] * kDq);
               const int col = h_row0(hc) + c0 + j;
               if (T::out_h) {
                 if (row_ok)
@@ -752,8 +784,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 16; k += 4) {
               float4 v;
               if (T::res)
-                v = make_float4(acc[j + k] * 0.00390625f, acc[j + k + 1] * 0.00390625f,
-                                acc[j + k + 2] * 0.00390625f, acc[j + k + 3] * 0.00390625f);
+                v = make_float4(acc[j + k] * kDq, acc[j + k + 1] * kDq,
+                                acc[j + k + 2] * kDq, acc[j + k + 3] * kDq);
               else
                 v = make_float4(lr[k], lr[k + 1], lr[k + 2], lr[k + 3]);
               *reinterpret_cast<float4*>(o + k) = v;
@@ -764,9 +796,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
               if (T::s2)
-                y[k] = acc[j + k] * 0.00390625f + lr[k];
+                y[k] = acc[j + k] * kDq + lr[k];
               else
-                y[k] = acc[j + k] * 0.00390625f;
+                y[k] = acc[j + k] * kDq;
             }
 #pragma unroll
             for (int k = 0; k < 16; k += 8) {
@@ -842,12 +874,12 @@ int num_sms() {
 
 // Clusters of two CTAs of the pair kernel that fit on the device at once, once
 // per instantiation (0 if the query fails: no pairs then).
-template <int kMode, int BN>
+template <int kMode, int BN, bool kA8>
 int resident_pairs() {
   static int cached = -1;
   if (cached < 0) {
-    using L = SmemLayout<BN>;
-    auto kern = twq_gemm_kernel<kMode, BN, true>;
+    using L = SmemLayout<BN, kA8>;
+    auto kern = twq_gemm_kernel<kMode, BN, true, kA8>;
     int nc = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) ==
         cudaSuccess) {
@@ -874,9 +906,9 @@ int resident_pairs() {
   return cached;
 }
 
-template <int kMode, int BN>
+template <int kMode, int BN, bool kA8 = false>
 cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
-  using L = SmemLayout<BN>;
+  using L = SmemLayout<BN, kA8>;
   using T = ModeTraits<kMode>;
   const twq_weights* w = c.w;
   GemmArgs a{};
@@ -900,7 +932,7 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
   bool pair = false;
   if constexpr (T::h && T::s2 && !T::h_global) {
     if (a.col_tiles % 2 == 0 && a.r % 32 == 0 && a.r > kHChunk && a.r <= 2 * kHChunk) {
-      const int pairs = resident_pairs<kMode, BN>();
+      const int pairs = resident_pairs<kMode, BN, kA8>();
       const int hc1 = (a.r + kHChunk - 1) / kHChunk;
       const int kc = (a.r + 63) / 64;
       const int n1 = a.row_blocks * a.col_tiles, n2 = a.row_blocks * (a.col_tiles / 2);
@@ -918,8 +950,11 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
 
   CUtensorMap m_xq{}, m_rq{}, m_l1q{}, m_l2t{}, m_h{};
   const uint64_t kb = static_cast<uint64_t>(a.m / 2);
-  bool ok = encode_2d(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, kb, c.b, kb, 64, kBM,
-                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  // W4A8: 128 int8 codes per row and group, with the 128-byte swizzle the MMA reads
+  bool ok = kA8 ? encode_2d(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, a.m, c.b, a.m, 128, kBM,
+                            CU_TENSOR_MAP_SWIZZLE_128B)
+                : encode_2d(&m_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.xq, kb, c.b, kb, 64, kBM,
+                            CU_TENSOR_MAP_SWIZZLE_NONE);
   if (T::res)
     ok = ok && encode_2d(&m_rq, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->rq, kb, a.n, kb, 64, BN,
                          CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -935,7 +970,7 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
   if (!ok) return cudaErrorInvalidValue;
 
   if (!pair || !(T::h && T::s2 && !T::h_global)) {
-    auto kern = twq_gemm_kernel<kMode, BN, false>;
+    auto kern = twq_gemm_kernel<kMode, BN, false, kA8>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
@@ -944,7 +979,7 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
     return cudaGetLastError();
   }
   if constexpr (T::h && T::s2 && !T::h_global) {
-  auto kern = twq_gemm_kernel<kMode, BN, true>;
+  auto kern = twq_gemm_kernel<kMode, BN, true, kA8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -960,7 +995,7 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // One wave of persistent pairs: as many as can be resident at once.
-  const int rp = resident_pairs<kMode, BN>();
+  const int rp = resident_pairs<kMode, BN, kA8>();
   const int pairs = a.num_tiles < rp ? a.num_tiles : rp;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
   e = cudaLaunchKernelEx(&cfg, kern, m_xq, m_rq, m_l1q, m_l2t, m_h, a);
@@ -974,10 +1009,13 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_gemm(const GemmCall& c, cudaStream_t st, int* launches) {
+  if (c.a8 && c.mode != kModeFused && c.mode != kModeW4A4) return cudaErrorInvalidValue;
   if (launches) ++*launches;
   switch (c.mode) {
-    case kModeFused: return launch_mode<kModeFused, 128>(c, st);
-    case kModeW4A4: return launch_mode<kModeW4A4, 128>(c, st);
+    case kModeFused:
+      return c.a8 ? launch_mode<kModeFused, 128, true>(c, st) : launch_mode<kModeFused, 128>(c, st);
+    case kModeW4A4:
+      return c.a8 ? launch_mode<kModeW4A4, 128, true>(c, st) : launch_mode<kModeW4A4, 128>(c, st);
     case kModeLowRank: return launch_mode<kModeLowRank, 128>(c, st);
     case kModeResF32: return launch_mode<kModeResF32, 128>(c, st);
     case kModeHOnly: return launch_mode<kModeHOnly, 128>(c, st);

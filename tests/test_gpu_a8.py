@@ -133,10 +133,31 @@ def test_w4a8_decode_workload(twq, device):
     _status_clean(twq)
 
 
-def test_w4a8_rejects_prefill_batches(twq, device):
-    x, R, L1, L2 = _operands(32, 1024, 256, 32, seed=2)
+PREFILL_SHAPES = [  # b > 16: the tensor-core GEMM kernel; ragged rows, two H chunks, r = 0,
+    # and CTA pairs (128 < r <= 256, even column-tile count)
+    (17, 384, 256, 64), (129, 512, 384, 128), (200, 256, 256, 144), (64, 640, 128, 0),
+    (300, 256, 1024, 256), (257, 384, 768, 160), (33, 1024, 512, 32),
+]
+
+
+@pytest.mark.parametrize("b,m,n,r", PREFILL_SHAPES)
+def test_w4a8_prefill_matches_oracle(twq, device, b, m, n, r):
+    x, R, L1, L2 = _operands(b, m, n, r, seed=43)
     w = _pack(twq, device, R, L1, L2)
-    xq8, sx = twq.quantize_act_a8(to_dev(x, device))
-    with pytest.raises(twq.TwqError) as e:
-        twq.fused_linear_a8(xq8, sx, w)
-    assert e.value.status == 2
+    y = bits_of(twq.fused_linear_a8(*twq.quantize_act_a8(to_dev(x, device)), w))
+    ref = oracle.layer(x, R, L1, L2, mode=oracle.FUSED if r else oracle.W4A4_ONLY, a8=True)["y"]
+    assert_y_close(y, ref, "W4A8 prefill %s" % ((b, m, n, r),))
+    _status_clean(twq)
+
+
+@pytest.mark.parametrize("name", ["gateup", "down"])
+def test_w4a8_prefill_workload_sampled_rows(twq, device, name):
+    wl = synth.WORKLOADS[name]
+    x = synth.make_x(wl, seed=5)
+    R, L1, L2 = synth.make_weights(wl, seed=5)
+    w = _pack(twq, device, R, L1, L2)
+    y = bits_of(twq.fused_linear_a8(*twq.quantize_act_a8(to_dev(x, device)), w))
+    rows = synth.sample_rows(wl.b, 12, seed=13)
+    ref = oracle.layer(x, R, L1, L2, rows=rows, a8=True)["y"]
+    assert_y_close(y[rows], ref, "W4A8 %s rows" % name)
+    _status_clean(twq)

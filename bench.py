@@ -542,9 +542,21 @@ def sweep(args, device, peaks):
             c = i % prob.copies
             twq.quantize_act(prob.x[c], prob.xq[c], prob.sx[c])
 
+        # W4A8: 8-bit activation codes for the same inputs (one buffer pair per copy)
+        xq8 = [torch.empty((b, wl.m), dtype=torch.int8, device=device) for _ in range(prob.copies)]
+        sx8 = [torch.empty_like(prob.sx[0]) for _ in range(prob.copies)]
+
+        def quant8(i):
+            c = i % prob.copies
+            twq.quantize_act_a8(prob.x[c], xq8[c], sx8[c])
+
+        def fused8(i):
+            c = i % prob.copies
+            twq.fused_linear_a8(xq8[c], sx8[c], prob.weights[c], prob.y[c])
 
         for i in range(prob.copies):
             quant(i)
+            quant8(i)
         torch.cuda.synchronize()
         t_f = kernel_only_time(prob, fused, steps, reps=3)
         t_w = kernel_only_time(prob, w4, steps, reps=3)
@@ -552,6 +564,7 @@ def sweep(args, device, peaks):
         t_q = kernel_only_time(prob, quant, steps, reps=3)
         t_x = kernel_only_time(prob, prob.step_x, steps, reps=3) if prob.one_launch else None
         t_a8 = kernel_only_time(prob, prob.step_x_a8, steps, reps=3) if prob.one_launch else None
+        t_f8 = kernel_only_time(prob, fused8, steps, reps=3)
         ops = int8_ops(b, wl.m, wl.n, wl.r) + bf16_flops(b, wl.n, wl.r)
         res.update({
             "fused_us": round(t_f * 1e6, 2), "w4a4_only_us": round(t_w * 1e6, 2),
@@ -560,6 +573,8 @@ def sweep(args, device, peaks):
             "lowrank_overhead": round(t_f / t_w - 1.0, 4), "fusion_speedup": round(t_u / t_f, 3),
             "roofline": roofline_entry(name, t_f, peaks, profiled_traffic(name)),
             "timing": "graph of back-to-back launches, weights rotating over %d copies" % prob.copies,
+            "w4a8_fused_us": round(t_f8 * 1e6, 2),
+            "w4a8_roofline": roofline_entry(name, t_f8, peaks, None),
         })
         if t_x is not None:
             res["fused_x_us"] = round(t_x * 1e6, 2)
@@ -568,7 +583,7 @@ def sweep(args, device, peaks):
             res["roofline_x"] = roofline_entry(name, t_x, peaks, profiled_traffic(name + "_x"),
                                                bf16_x=True)
         out.append(res)
-        del prob, ws
+        del prob, ws, xq8, sx8
         torch.cuda.empty_cache()
     out.append(fold_entry(device))
     st = twq.device_status()

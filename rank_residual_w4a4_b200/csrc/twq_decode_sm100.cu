@@ -28,6 +28,7 @@
 // reads a peer's shared memory, and every write into it has landed once its
 // bounded wait completes, so no CTA exits while a peer may still write into it.
 #include <atomic>
+#include <mutex>
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
@@ -742,9 +743,59 @@ EncodeTiledFn d_encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps by their parameters. A decode call is short, so the host
+// cost of encoding its four maps matters; the weights' maps repeat on every call
+// of a layer. A map only encodes an address and a shape, so a hit is exact.
+struct MapKey {
+  const void* base;
+  uint64_t inner, outer, row_bytes;
+  uint32_t box_inner, box_outer;
+  int dt, sw;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+           box_inner == o.box_inner && box_outer == o.box_outer && dt == o.dt && sw == o.sw;
+  }
+};
+constexpr int kMapCacheSize = 256;  // direct-mapped
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+MapEntry g_map_cache[kMapCacheSize];
+std::mutex g_map_mutex;
+
+bool d_encode_raw(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle sw);
+
 bool d_encode(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
               CUtensorMapSwizzle sw) {
+  const MapKey key{base, inner, outer, row_bytes, box_inner, box_outer, static_cast<int>(dt),
+                   static_cast<int>(sw)};
+  uint64_t h = reinterpret_cast<uintptr_t>(base) * 0x9E3779B97F4A7C15ull;
+  h ^= (inner * 31 + outer) * 0xC2B2AE3D27D4EB4Full;
+  h ^= (row_bytes + (uint64_t(box_inner) << 20) + (uint64_t(box_outer) << 40) + key.dt * 7 + key.sw);
+  MapEntry& e = g_map_cache[(h >> 32) % kMapCacheSize];
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    if (e.valid && e.key == key) {
+      *map = e.map;
+      return true;
+    }
+  }
+  if (!d_encode_raw(map, dt, base, inner, outer, row_bytes, box_inner, box_outer, sw)) return false;
+  std::lock_guard<std::mutex> lock(g_map_mutex);
+  e.key = key;
+  e.map = *map;
+  e.valid = true;
+  return true;
+}
+
+bool d_encode_raw(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle sw) {
   EncodeTiledFn fn = d_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};

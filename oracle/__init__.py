@@ -254,3 +254,32 @@ def fold_transforms(Q, G, U, V, R, rounded=True):
     if not rounded:
         return l1, l2, rr
     return _f64_to_bf16(l1), _f64_to_bf16(l2), _f64_to_bf16(rr)
+
+
+def layer_s2q(x_bits, R, L1, L2, rows=None, want=("y",)):
+    """The layer with the pages' INT4 stage 2 (TwinQuant §4.3: H is requantized to
+    4 bits on chip and multiplied by the 4-bit V). Readings: H is first rounded to
+    BF16 (as in the BF16 stage 2); Q_H is Eq. (1) on it per token in groups of 128
+    along r; V = L2 is quantized per output column in groups of 128 along r; both
+    with q_max = 7. Then, per group g of r (Eq. (2) applied group by group):
+
+        Y_lr[i, j] = sum_g sH[i, g] * sV[g, j] * sum_{k in g} qH[i, k] * qV[j, k]
+        Y          = bf16(float(Y_res + Y_lr))
+
+    Needs r % 128 == 0. Returns a dict of the wanted outputs among y (BF16 bits),
+    y64 (float64), hb (BF16 bits of H), qh, sh (codes and scales of H)."""
+    qx, sx = quantize_rows(x_bits)
+    qr, sr = quantize_cols(R)
+    ql1, sl1 = quantize_cols(L1)
+    r = ql1.shape[0]
+    if r % GROUP:
+        raise ValueError("the INT4 stage 2 needs r % 128 == 0")
+    res = linear(qx, sx, qr, sr, None, None, None, mode=W4A4_ONLY, rows=rows, want=("y64",))["y64"]
+    hb = linear(qx, sx, None, None, ql1, sl1, L2, mode=LOWRANK_ONLY, rows=rows, want=("hb",))["hb"]
+    qh, sh = quantize_rows(hb)          # Eq. (1) on bf16(H), per token, groups of 128 along r
+    qv, sv = quantize_cols(L2)          # Eq. (1) on L2 (r x n), per column, groups along r
+    # the grouped integer GEMM of Eq. (2), with qH as the activations and qV as the weights
+    ylr = linear(qh, sh, qv, sv, None, None, None, mode=W4A4_ONLY, want=("y64",))["y64"]
+    total = res + ylr
+    out = {"y": _f64_to_bf16(total), "y64": total, "hb": hb, "qh": qh, "sh": sh}
+    return {k: out[k] for k in want}

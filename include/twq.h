@@ -219,6 +219,31 @@ TWQ_API twq_status twq_fused_linear_a8(const int8_t* xq8, const float* sx, int64
 TWQ_API twq_status twq_fused_linear_x_a8(const uint16_t* x, int64_t ldx, int64_t b,
                                          const twq_weights* w, uint16_t* y, twq_stream_t stream);
 
+/*
+ * The INT4 stage 2 of TwinQuant §4.3 (H requantized on chip to 4 bits and
+ * multiplied by a 4-bit V = L2). Readings: H is rounded to BF16 as in the BF16
+ * stage 2, then quantized with Eq. (1) (q_max = 7) per token in groups of 128
+ * along r; L2 is quantized per output column in groups of 128 along r. Stage 2 is
+ * then Eq. (2) group by group:
+ *     Y = bf16(Y_res + sum_g s_H[i,g] s_V[g,j] sum_{k in g} Q_H[i,k] Q_V[j,k])
+ * Limits: r == 128 or r == 256.
+ *
+ * twq_pack_l2_int4: L2 (r x n BF16, row-major) -> l2q (n x r/2 bytes, column j of
+ *   L2 contiguous along r, nibbles as the codes format above) and sl2q ((r/128) x n
+ *   fp32). Offline, with twq_pack_weights; bit-exact.
+ * twq_fused_linear_s2q: xq, sx from twq_quantize_act; w from twq_pack_weights (its
+ *   l2t is not read); l2q, sl2q from twq_pack_l2_int4; y b x n BF16. One launch of
+ *   the tensor-core GEMM kernel for any b (H never leaves the chip; its codes
+ *   overwrite it in shared memory and feed r/128 more int8 K groups of the residual
+ *   accumulation). Errors as twq_fused_linear; r outside {128, 256} returns
+ *   TWQ_ERR_UNSUPPORTED (r == 0: TWQ_ERR_INVALID_ARG).
+ */
+TWQ_API twq_status twq_pack_l2_int4(const uint16_t* L2, int64_t r, int64_t n, uint8_t* l2q,
+                                    float* sl2q, twq_stream_t stream);
+TWQ_API twq_status twq_fused_linear_s2q(const uint8_t* xq, const float* sx, int64_t b,
+                                        const twq_weights* w, const uint8_t* l2q,
+                                        const float* sl2q, uint16_t* y, twq_stream_t stream);
+
 /* Residual component only: Y = bf16(Q(X) Q(R)) (TwinQuant Eq. (2)); ignores l1q/sl1/l2t. */
 TWQ_API twq_status twq_w4a4_only(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
                          uint16_t* y, twq_stream_t stream);

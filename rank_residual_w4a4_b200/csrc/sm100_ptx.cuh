@@ -24,6 +24,8 @@ enum WaitSite : int {
   kSiteFinal = 10,
   kSiteProducerHbFree = 11,
   kSiteDrainPeerFree = 12,
+  kSiteDrainHq = 13,   // the drain warps' BF16 H (INT4 stage 2)
+  kSiteDrainHbq = 14,  // the requantized H and its scales (INT4 stage 2)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

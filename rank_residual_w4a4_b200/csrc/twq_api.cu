@@ -170,6 +170,31 @@ twq_status twq_fused_linear_a8(const int8_t* xq8, const float* sx, int64_t b, co
   return from_cuda(twq::launch_gemm(c, st, nullptr));
 }
 
+twq_status twq_pack_l2_int4(const uint16_t* L2, int64_t r, int64_t n, uint8_t* l2q, float* sl2q,
+                            twq_stream_t stream) {
+  if (r <= 0 || r % 128 || n <= 0 || n % 128) return TWQ_ERR_INVALID_ARG;
+  if (r > 256 || n > (int64_t(1) << 24)) return TWQ_ERR_UNSUPPORTED;
+  if (!L2 || !l2q || !sl2q) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(L2) || !aligned16(l2q) || !aligned16(sl2q)) return TWQ_ERR_MISALIGNED;
+  return from_cuda(twq::launch_pack_cols(L2, r, n, l2q, sl2q, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+twq_status twq_fused_linear_s2q(const uint8_t* xq, const float* sx, int64_t b, const twq_weights* w,
+                                const uint8_t* l2q, const float* sl2q, uint16_t* y,
+                                twq_stream_t stream) {
+  if (!w) return TWQ_ERR_INVALID_ARG;
+  if (w->r <= 0 || w->r % 128) return w->r > 0 ? TWQ_ERR_UNSUPPORTED : TWQ_ERR_INVALID_ARG;
+  twq_status s = check_layer(xq, sx, b, w, y, true, false);
+  if (s != TWQ_OK || b == 0) return s;
+  if (!w->l1q || !w->sl1 || !l2q || !sl2q) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(w->l1q) || !aligned16(w->sl1) || !aligned16(l2q) || !aligned16(sl2q))
+    return TWQ_ERR_MISALIGNED;
+  twq::GemmCall c{twq::kModeFusedS2Q, xq, sx, b, w, y, nullptr};
+  c.l2q = l2q;
+  c.sl2q = sl2q;
+  return from_cuda(twq::launch_gemm(c, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
 // Validates a twq_fused_linear_x call (b >= 1) and fills the decode launch.
 static twq_status prepare_fused_x(const uint16_t* x, int64_t ldx, int64_t b, const twq_weights* w,
                                   uint16_t* y, twq::GemmCall* out, bool a8 = false) {
@@ -282,6 +307,7 @@ int twq_launches_per_call(const char* ep) {
   if (!ep) return -1;
   if (!strcmp(ep, "twq_quantize_act") || !strcmp(ep, "twq_quantize_act_a8")) return 1;
   if (!strcmp(ep, "twq_pack_weights")) return 3;
+  if (!strcmp(ep, "twq_pack_l2_int4") || !strcmp(ep, "twq_fused_linear_s2q")) return 1;
   if (!strcmp(ep, "twq_fused_linear") || !strcmp(ep, "twq_w4a4_only") ||
       !strcmp(ep, "twq_lowrank_only") || !strcmp(ep, "twq_fused_linear_x") ||
       !strcmp(ep, "twq_fused_linear_x_host") || !strcmp(ep, "twq_fused_linear_a8") ||

@@ -169,15 +169,6 @@ __device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int j, uin
 // the codes are identical (the group maximum is exact in any order).
 constexpr int kQPairsPerPass = 80;  // 10 warps x 8 pairs
 
-__device__ __forceinline__ uint4 pack_codes16(const uint32_t (&nb)[16]) {
-  // 16*q bytes: even elements 0..6, odd 1..7, even 8..14, odd 9..15
-  uint4 o;
-  o.x = (nb[0] << 4) | (nb[1] << 12) | (nb[2] << 20) | (nb[3] << 28);
-  o.y = (nb[8] << 4) | (nb[9] << 12) | (nb[10] << 20) | (nb[11] << 28);
-  o.z = (nb[4] << 4) | (nb[5] << 12) | (nb[6] << 20) | (nb[7] << 28);
-  o.w = (nb[12] << 4) | (nb[13] << 12) | (nb[14] << 20) | (nb[15] << 28);
-  return o;
-}
 
 // 16 int8 codes (q_max = 127) in the same in-chunk order as pack_codes16.
 __device__ __forceinline__ uint4 pack_codes16_a8(const uint32_t (&c)[16]) {

@@ -94,6 +94,18 @@ __device__ __forceinline__ void eq1_codes(const float (&v)[N], const Eq1Scale& k
   }
 }
 
+// Sixteen 4-bit codes of one 16-element chunk (nb[0..7]: even elements 0, 2, .., 14;
+// nb[8..15]: odd elements) as int8 bytes 16*q in the MMA operand order the 4-bit
+// unpack produces: even elements 0..6, odd 1..7, even 8..14, odd 9..15.
+__device__ __forceinline__ uint4 pack_codes16(const uint32_t (&nb)[16]) {
+  uint4 o;
+  o.x = (nb[0] << 4) | (nb[1] << 12) | (nb[2] << 20) | (nb[3] << 28);
+  o.y = (nb[8] << 4) | (nb[9] << 12) | (nb[10] << 20) | (nb[11] << 28);
+  o.z = (nb[4] << 4) | (nb[5] << 12) | (nb[6] << 20) | (nb[7] << 28);
+  o.w = (nb[12] << 4) | (nb[13] << 12) | (nb[14] << 20) | (nb[15] << 28);
+  return o;
+}
+
 template <int N>
 __device__ __forceinline__ void eq1_nibbles(const float (&v)[N], const Eq1Scale& k,
                                             uint32_t (&nib)[N]) {

@@ -30,6 +30,7 @@
 #include <algorithm>
 
 #include "sm100_ptx.cuh"
+#include "twq_eq1.cuh"
 #include "twq_internal.h"
 
 namespace twq {
@@ -51,8 +52,13 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a wait that lasts 2 s is a 
 
 template <int kMode>
 struct ModeTraits {
-  static constexpr bool res = kMode == kModeFused || kMode == kModeW4A4 || kMode == kModeResF32;
-  static constexpr bool h = kMode == kModeFused || kMode == kModeLowRank || kMode == kModeHOnly;
+  static constexpr bool res = kMode == kModeFused || kMode == kModeW4A4 || kMode == kModeResF32 ||
+                              kMode == kModeFusedS2Q;
+  static constexpr bool h = kMode == kModeFused || kMode == kModeLowRank || kMode == kModeHOnly ||
+                            kMode == kModeFusedS2Q;
+  // The INT4 stage 2: H requantized on chip, multiplied by 4-bit L2 codes as r/128 more
+  // K groups of the residual accumulation (kind::i8), not by the BF16 stage 2.
+  static constexpr bool s2q = kMode == kModeFusedS2Q;
   static constexpr bool s2 = kMode == kModeFused || kMode == kModeLowRank || kMode == kModeS2F32;
   static constexpr bool h_global = kMode == kModeS2F32;
   static constexpr bool out_f32 = kMode == kModeResF32 || kMode == kModeS2F32;
@@ -76,9 +82,10 @@ struct SmemLayout {
   static constexpr int kOffU = kOffSlots + kStages * kSlot;
   static constexpr int kOffHb = kOffU + kUnpackedStages * kUStage;
   static constexpr int kOffScale = kOffHb + kHb;
-  static constexpr int kOffBar = kOffScale + kScaleSlots * kScaleSlot;
+  static constexpr int kOffShq = kOffScale + kScaleSlots * kScaleSlot;  // s_H: 128 rows x 2 groups
+  static constexpr int kOffBar = kOffShq + kBM * 2 * 4;
   static constexpr int kNumBars =
-      2 * kStages + 2 * kUnpackedStages + 2 * kAccBufs + 2 * kScaleSlots + 4;
+      2 * kStages + 2 * kUnpackedStages + 2 * kAccBufs + 2 * kScaleSlots + 5;
   static constexpr int kBytes = kOffBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
   static constexpr int kTmemCols = kAccBufs * BN;  // accumulator buffers
@@ -98,6 +105,7 @@ struct GemmArgs {
   int tiles_per_rb;  // tiles (or, for CTA pairs, pairs of column tiles) per row block
   int r_pad;  // stage-2 K extent: r rounded up to 64
   int h_box;  // rows of the L1 TMA box: min(r, 128)
+  const float* sl2q;  // INT4 stage 2: scales of the 4-bit L2 codes, (r/128) x n
 };
 
 struct Ring {
@@ -293,6 +301,49 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, int t, int t_be
   return ti;
 }
 
+// Eq. (1) (q_max = 7) on one row of a group of 128 BF16 columns of H in the stage-2
+// operand layout (two 16 KB chunks of 64 columns, 128-byte swizzle, starting at `grp`),
+// written back as 16*q int8 codes in the 4-bit operand order over the first chunk.
+// Piece p (columns [8p, 8p + 8)) sits at location p; output chunk c (columns
+// [16c, 16c + 16)) reads pieces 2c and 2c + 1 and is written at location c, which
+// holds piece c, already read by output chunk c / 2 <= c: in place, in one stream.
+__device__ __forceinline__ const uint4* h_piece(const uint8_t* grp, int row, int p) {
+  return reinterpret_cast<const uint4*>(grp + (p >> 3) * 16384 + sw128_offset(row, p & 7));
+}
+
+__device__ __noinline__ void requant_h_row(uint8_t* grp, int row, float* s_out) {
+  float a = 0.0f;
+#pragma unroll 4
+  for (int p = 0; p < 16; ++p) {
+    const uint4 w = *h_piece(grp, row, p);
+    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      a = fmaxf(a, fmaxf(fabsf(__uint_as_float(v[i] << 16)),
+                         fabsf(__uint_as_float(v[i] & 0xFFFF0000u))));
+  }
+  const Eq1Scale ks = eq1_scale<7>(a);
+  *s_out = ks.s;
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (ks.s != 0.0f) {
+      const uint4 w0 = *h_piece(grp, row, 2 * c), w1 = *h_piece(grp, row, 2 * c + 1);
+      const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      float f[16];  // f[0..7]: even columns 0, 2, .., 14 of the chunk; f[8..15]: odd
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        f[i] = __uint_as_float(u[i] << 16);
+        f[8 + i] = __uint_as_float(u[i] & 0xFFFF0000u);
+      }
+      uint32_t nb[16];
+      eq1_nibbles(f, ks, nb);
+      o = pack_codes16(nb);
+    }
+    *reinterpret_cast<uint4*>(grp + sw128_offset(row, c)) = o;
+  }
+}
+
 // kPair: a cluster of two CTAs works on the two column tiles of one pair at a
 // time; CTA k computes H columns [k r/2, (k+1) r/2) of the row block and stores
 // its BF16 slice into both CTAs' H operand tiles, so H is computed once per pair.
@@ -330,7 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* hb_free = hb_ready + 1;
   uint64_t* mma_done = hb_free + 1;
   uint64_t* peer_free = mma_done + 1;  // kPair: the peer may overwrite its slice of our H
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
+  uint64_t* hq = mma_done + 2;         // INT4 stage 2: every drain warp's BF16 H is in hb
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 3);
+  float* shq = reinterpret_cast<float*>(smem + L::kOffShq);  // s_H[row * 2 + group of r]
   volatile int* abort_flag = &s_abort;
 
   const int warp = threadIdx.x >> 5;
@@ -365,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(hb_free, 1);
     mbar_init(mma_done, 1);
     mbar_init(peer_free, 1);
+    mbar_init(hq, 8);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -466,6 +520,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             q.next(kScaleSlots);
           }
         }
+        if (T::s2q && ok) {
+          // INT4 stage 2: the tile's 4-bit L2 codes, one group of 128 along r per step
+          // (the A operand, the requantized H, is already on chip), and their scales
+          for (int g2 = 0; g2 < args.r / 128; ++g2) {
+            if (!(ok = wait_fast(&empty[s.idx], s.phase ^ 1u, abort_flag, kSiteProducerEmpty)))
+              break;
+            uint8_t* slot = slots + s.idx * L::kSlot;
+            mbar_arrive_expect_tx(&full[s.idx], BN * 64);
+            tma_load_2d(slot + L::kSlotA, &tm_l2t, &full[s.idx], g2 * 64, n0);
+            pend[s.idx] = true;
+            pend_phase[s.idx] = s.phase;
+            s.next(kStages);
+            if (!(ok = wait_fast(&sc_empty[q.idx], q.phase ^ 1u, abort_flag,
+                                kSiteProducerScaleEmpty)))
+              break;
+            mbar_arrive_expect_tx(&sc_full[q.idx], BN * 4);
+            bulk_load(scl + q.idx * BN, args.sl2q + (int64_t)g2 * args.n + n0, BN * 4,
+                      &sc_full[q.idx]);
+            spend[q.idx] = true;
+            spend_phase[q.idx] = q.phase;
+            q.next(kScaleSlots);
+          }
+        }
         if (T::s2 && ok) {
           if (T::h_global) {
             if (!(ok = wait_fast(hb_free, hb_phase ^ 1u, abort_flag, kSiteProducerHbFree))) break;
@@ -556,6 +633,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             a.next(kAccBufs);
           }
         }
+        if (T::s2q && ok) {
+          // INT4 stage 2: A = the requantized H of group g2 (int8 16*q, written by the
+          // drain warps over the first 16 KB of H's BF16 columns [128 g2, 128 g2 + 128)),
+          // B = the unpacked 4-bit L2 codes
+          if (ti.need_h) {
+            if (!(ok = wait_fast(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) break;
+            hb_phase ^= 1u;
+          }
+          const uint32_t idesc = idesc_i8(BN);
+          for (int g2 = 0; g2 < args.r / 128; ++g2) {
+            if (!(ok = wait_fast(&ufull[u.idx], u.phase, abort_flag, kSiteMmaFull))) break;
+            if (!(ok = wait_fast(&acc_empty[a.idx], a.phase ^ 1u, abort_flag, kSiteMmaAccEmpty)))
+              break;
+            tc_fence_after();
+            const uint32_t d = tmem_base + a.idx * BN;
+            const uint64_t da = smem_desc_sw128(hb0 + g2 * 32768);
+            const uint64_t db = smem_desc_sw128(ua0 + u.idx * L::kUStage + L::kUA);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mma_i8(d, da + 2 * k, db + 2 * k, idesc, k > 0);
+            mma_commit(&uempty[u.idx]);
+            mma_commit(&acc_full[a.idx]);
+            release_slot();
+            u.next(kUnpackedStages);
+            a.next(kAccBufs);
+          }
+        }
         if (T::s2 && ok) {
           if (ti.need_h || T::h_global) {
             if (kPair) {
@@ -605,8 +708,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileInfo ti = tile_info(args, t, t_begin, T::h, kPairStride, prank);
       const int n_h = ti.need_h ? HC * G : 0;
       const int n_res = T::res ? G : 0;
+      const int n_q = T::s2q ? args.r / 128 : 0;
       const int n_l2 = T::s2 ? KC : 0;
-      for (int step = 0; step < n_h + n_res + n_l2; ++step) {
+      for (int step = 0; step < n_h + n_res + n_q + n_l2; ++step) {
         if (!(ok = wait_bar(&full[s.idx], s.phase, abort_flag, kSiteUnpackFull))) break;
         if (!(ok = wait_bar(&uempty[u.idx], u.phase ^ 1u, abort_flag, kSiteUnpackEmpty))) break;
         const uint8_t* src = slots + s.idx * L::kSlot;
@@ -619,6 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if constexpr (!kA8) unpack_tile(src, dst, kBM, plan);  // W4A8: the MMA reads X in place
           unpack_tile<kA8>(src + L::kSlotA, dst + L::kUA, brows, plan);
+        } else if (step < n_h + n_res + n_q) {  // INT4 stage 2: only the L2 codes (B)
+          unpack_tile(src + L::kSlotA, dst + L::kUA, BN, plan);
         } else {
           copy_smem(src, dst + L::kUA, BN * 128, tid, 192);
         }
@@ -641,6 +747,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     Ring a, q;
     uint32_t peer_phase = 0;  // kPair: phase of peer_free for the next H slice
+    uint32_t hq_phase = 0;    // INT4 stage 2: phases of hq and (as a consumer) of hb_ready
+    uint32_t hbq_phase = 0;
     bool ok = true;
     float acc[64];
     for (int t = t_begin; t < t_end && ok; ++t) {
@@ -716,6 +824,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
+        if constexpr (T::s2q) {
+          // INT4 stage 2: Eq. (1) on bf16(H) per row and group of 128 along r. A group's
+          // columns come from both halves' warps, so every drain warp's BF16 H must be in
+          // hb first (a bounded barrier, so that an aborting warp cannot strand the others).
+          __syncwarp();
+          if (lane == 0) mbar_arrive(hq);
+          if (!(ok = wait_bar(hq, hq_phase, abort_flag, kSiteDrainHq))) break;
+          hq_phase ^= 1u;
+          // Thread (row, half) takes group `half` of its row: it reads the group's 128 BF16
+          // values (16 pieces of 8) into registers, then writes the 16*q codes over the
+          // group's first 16 KB (only this thread touches these bytes of this row).
+          if (half < args.r / 128) requant_h_row(hb + half * 32768, row_in, shq + row_in * 2 + half);
+        }
         if (!T::out_h) {
           fence_proxy_async_smem();
           __syncwarp();
@@ -746,6 +867,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(&sc_full[q.idx], q.phase, abort_flag, kSiteDrainScaleFull))) break;
           drain_group(acc, tmem_base + lane_addr + a.idx * BN + c0, ncols, scl + q.idx * BN + c0,
                       sx);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&acc_empty[a.idx]);
+            mbar_arrive(&sc_empty[q.idx]);
+          }
+          a.next(kAccBufs);
+          q.next(kScaleSlots);
+        }
+        if (!ok) break;
+      }
+      if (T::s2q) {
+        // INT4 stage 2 as r/128 more groups of the same accumulation: I * s_V[col] * s_H[row]
+        if (ti.need_h) {  // the requantized H and its scales are complete
+          if (!(ok = wait_bar(hb_ready, hbq_phase, abort_flag, kSiteDrainHbq))) break;
+          hbq_phase ^= 1u;
+        }
+        for (int g2 = 0; g2 < args.r / 128; ++g2) {
+          const float sh = shq[row_in * 2 + g2];
+          if (!(ok = wait_bar(&acc_full[a.idx], a.phase, abort_flag, kSiteDrainAccFull))) break;
+          tc_fence_after();
+          if (!(ok = wait_bar(&sc_full[q.idx], q.phase, abort_flag, kSiteDrainScaleFull))) break;
+          drain_group(acc, tmem_base + lane_addr + a.idx * BN + c0, ncols, scl + q.idx * BN + c0,
+                      sh);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
@@ -964,6 +1109,12 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
   if (T::s2)
     ok = ok && encode_2d(&m_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2t, a.r, a.n,
                          static_cast<uint64_t>(a.r) * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (T::s2q) {  // the 4-bit L2 codes: n rows of r/2 bytes, 64 bytes (128 codes) per group
+    a.sl2q = c.sl2q;
+    ok = ok && c.l2q && c.sl2q &&
+         encode_2d(&m_l2t, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.l2q, a.r / 2, a.n,
+                   static_cast<uint64_t>(a.r / 2), 64, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
   if (T::h_global)
     ok = ok && encode_2d(&m_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.h_global, a.r, c.b,
                          static_cast<uint64_t>(a.r) * 2, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -1020,6 +1171,7 @@ cudaError_t launch_gemm(const GemmCall& c, cudaStream_t st, int* launches) {
     case kModeResF32: return launch_mode<kModeResF32, 128>(c, st);
     case kModeHOnly: return launch_mode<kModeHOnly, 128>(c, st);
     case kModeS2F32: return launch_mode<kModeS2F32, 128>(c, st);
+    case kModeFusedS2Q: return launch_mode<kModeFusedS2Q, 128>(c, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -16,6 +16,7 @@ enum GemmMode : int {
   kModeResF32 = 3,   // out = Q(X)Q(R) in fp32            (unfused comparator, step 1)
   kModeHOnly = 4,    // out = bf16(Q(X)Q(L1)), b x r      (unfused comparator, step 2)
   kModeS2F32 = 5,    // out = H L2 in fp32, H read from HBM (unfused comparator, step 3)
+  kModeFusedS2Q = 6, // Y = bf16(Q(X)Q(R) + Q(bf16(Q(X)Q(L1))) Q(L2)): the INT4 stage 2
 };
 
 struct GemmCall {
@@ -28,7 +29,9 @@ struct GemmCall {
   const uint16_t* h_global; // kModeS2F32 only: bf16 H, b x r
   const uint16_t* x = nullptr;  // decode kernel only: BF16 X, quantized in the kernel
   int64_t ldx = 0;
-  bool a8 = false;  // W4A8 (decode kernel only): xq holds int8 codes (q_max = 127), b x m
+  bool a8 = false;  // W4A8: xq holds int8 codes (q_max = 127), b x m
+  const uint8_t* l2q = nullptr;  // kModeFusedS2Q: L2 as 4-bit codes, n x r/2 (K-major)
+  const float* sl2q = nullptr;   // kModeFusedS2Q: their scales, (r/128) x n
 };
 
 // Host-side launchers; all return cudaSuccess or the launch error.

@@ -29,7 +29,7 @@ EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_siz
            "twq_device_status", "twq_launches_per_call", "twq_unfused_linear_noalloc",
            "twq_fused_linear_x", "twq_fold_workspace_bytes", "twq_fold_transforms",
            "twq_fused_linear_x_host", "twq_quantize_act_a8", "twq_fused_linear_a8",
-           "twq_fused_linear_x_a8")
+           "twq_fused_linear_x_a8", "twq_pack_l2_int4", "twq_fused_linear_s2q")
 
 
 class TwqError(RuntimeError):
@@ -77,6 +77,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twq_quantize_act_a8": ([P, I, I, I, P, P, P], ctypes.c_int),
         "twq_fused_linear_a8": ([P, P, I, P, P, P], ctypes.c_int),
         "twq_fused_linear_x_a8": ([P, I, I, P, P, P], ctypes.c_int),
+        "twq_pack_l2_int4": ([P, I, I, P, P, P], ctypes.c_int),
+        "twq_fused_linear_s2q": ([P, P, I, P, P, P, P, P], ctypes.c_int),
         "twq_fold_workspace_bytes": ([I, I, I], S),
         "twq_fold_transforms": ([P, P, P, P, P, I, I, I, P, P, P, P, S, P], ctypes.c_int),
     }
@@ -231,6 +233,32 @@ def fused_linear_a8(xq8, sx, w: Weights, y=None, stream=None):
     _check(load().twq_fused_linear_a8(_dev(xq8, "xq8", torch.int8), _dev(sx, "sx", torch.float32),
                                       b, ctypes.byref(cw), _dev(y, "y", torch.bfloat16),
                                       _stream(stream)), "twq_fused_linear_a8")
+    return y
+
+
+def pack_l2_int4(L2: torch.Tensor, stream=None):
+    """The INT4 stage 2's V: BF16 L2 (r x n) -> 4-bit codes (n x r/2 uint8) and scales
+    ((r/128) x n fp32), groups of 128 along r per output column."""
+    r, n = L2.shape
+    l2q = torch.empty((n, r // 2), dtype=torch.uint8, device=L2.device)
+    sl2q = torch.empty((max(r // 128, 1), n), dtype=torch.float32, device=L2.device)
+    _check(load().twq_pack_l2_int4(_dev(L2, "L2", torch.bfloat16), r, n,
+                                   _dev(l2q, "l2q", torch.uint8), _dev(sl2q, "sl2q", torch.float32),
+                                   _stream(stream)), "twq_pack_l2_int4")
+    return l2q, sl2q
+
+
+def fused_linear_s2q(xq, sx, w: Weights, l2q, sl2q, y=None, stream=None):
+    """The fused layer with the INT4 stage 2 (H requantized on chip, 4-bit L2)."""
+    b = xq.shape[0]
+    if y is None:
+        y = torch.empty((b, w.n), dtype=torch.bfloat16, device=xq.device)
+    cw = w.c_struct()
+    _check(load().twq_fused_linear_s2q(_dev(xq, "xq", torch.uint8), _dev(sx, "sx", torch.float32),
+                                       b, ctypes.byref(cw), _dev(l2q, "l2q", torch.uint8),
+                                       _dev(sl2q, "sl2q", torch.float32),
+                                       _dev(y, "y", torch.bfloat16), _stream(stream)),
+           "twq_fused_linear_s2q")
     return y
 
 

@@ -164,6 +164,24 @@ def test_w4a8_validation(lib):
     assert fx(A, 512, 0, ctypes.byref(w), None, None) == 0
 
 
+def test_s2q_validation(lib):
+    # every rejection happens before anything is launched
+    pk = lib.twq_pack_l2_int4
+    assert pk(None, 128, 256, A, A, None) == 1
+    assert pk(A, 96, 256, A, A, None) == 1      # r % 128
+    assert pk(A, 128, 200, A, A, None) == 1     # n % 128
+    assert pk(A, 384, 256, A, A, None) == 2     # r > 256
+    assert pk(A + 2, 128, 256, A, A, None) == 3
+    f = lib.twq_fused_linear_s2q
+    w = _w(r=128)
+    assert f(A, A, 4, None, A, A, A, None) == 1
+    assert f(A, A, 4, ctypes.byref(_w(r=0)), A, A, A, None) == 1
+    assert f(A, A, 4, ctypes.byref(_w(r=64)), A, A, A, None) == 2
+    assert f(A, A, 4, ctypes.byref(w), None, A, A, None) == 1
+    assert f(A, A, 4, ctypes.byref(w), A + 4, A, A, None) == 3
+    assert f(A, A, 0, ctypes.byref(w), A, A, None, None) == 0
+
+
 def test_fold_validation(lib):
     f = lib.twq_fold_transforms
     ws = lib.twq_fold_workspace_bytes(256, 128, 32)
@@ -207,7 +225,8 @@ def test_launch_accounting(lib):
     assert twq.launches_per_call("twq_unfused_linear_noalloc") == 4
     assert twq.launches_per_call("twq_fused_linear_x") == 1
     assert twq.launches_per_call("twq_fused_linear_x_host") == 1
-    for ep in ("twq_quantize_act_a8", "twq_fused_linear_a8", "twq_fused_linear_x_a8"):
+    for ep in ("twq_quantize_act_a8", "twq_fused_linear_a8", "twq_fused_linear_x_a8",
+               "twq_pack_l2_int4", "twq_fused_linear_s2q"):
         assert twq.launches_per_call(ep) == 1
     assert twq.launches_per_call("twq_fold_transforms") == 5
     assert twq.launches_per_call("nope") == -1

@@ -554,6 +554,15 @@ def sweep(args, device, peaks):
             c = i % prob.copies
             twq.fused_linear_a8(xq8[c], sx8[c], prob.weights[c], prob.y[c])
 
+        # the INT4 stage 2 (r = 128 or 256): 4-bit L2 codes per weight copy
+        s2q = wl.r in (128, 256)
+        l2qs = [twq.pack_l2_int4(wc.l2t.t().contiguous()) for wc in prob.weights] if s2q else []
+
+        def fused_s2q(i):
+            c = i % prob.copies
+            twq.fused_linear_s2q(prob.xq[c], prob.sx[c], prob.weights[c], l2qs[c][0], l2qs[c][1],
+                                 prob.y[c])
+
         for i in range(prob.copies):
             quant(i)
             quant8(i)
@@ -565,6 +574,7 @@ def sweep(args, device, peaks):
         t_x = kernel_only_time(prob, prob.step_x, steps, reps=3) if prob.one_launch else None
         t_a8 = kernel_only_time(prob, prob.step_x_a8, steps, reps=3) if prob.one_launch else None
         t_f8 = kernel_only_time(prob, fused8, steps, reps=3)
+        t_s2q = kernel_only_time(prob, fused_s2q, steps, reps=3) if s2q else None
         ops = int8_ops(b, wl.m, wl.n, wl.r) + bf16_flops(b, wl.n, wl.r)
         res.update({
             "fused_us": round(t_f * 1e6, 2), "w4a4_only_us": round(t_w * 1e6, 2),
@@ -576,6 +586,8 @@ def sweep(args, device, peaks):
             "w4a8_fused_us": round(t_f8 * 1e6, 2),
             "w4a8_roofline": roofline_entry(name, t_f8, peaks, None),
         })
+        if t_s2q is not None:
+            res["s2q_fused_us"] = round(t_s2q * 1e6, 2)
         if t_x is not None:
             res["fused_x_us"] = round(t_x * 1e6, 2)
             res["fused_x_a8_us"] = round(t_a8 * 1e6, 2)
@@ -583,7 +595,7 @@ def sweep(args, device, peaks):
             res["roofline_x"] = roofline_entry(name, t_x, peaks, profiled_traffic(name + "_x"),
                                                bf16_x=True)
         out.append(res)
-        del prob, ws, xq8, sx8
+        del prob, ws, xq8, sx8, l2qs
         torch.cuda.empty_cache()
     out.append(fold_entry(device))
     st = twq.device_status()

@@ -21,7 +21,8 @@
 //   GEMM and the first low-rank GEMM; the first stage's result H is
 //   converted and fed to the second stage; a single epilogue adds both parts.
 //   In this build the second stage takes H rounded to BF16 and L2 in BF16
-//   (not the page's on-the-fly INT4 requantization), and Y is BF16.
+//   (the page's on-the-fly INT4 requantization is composed from these functions
+//   in oracle.layer_s2q), and Y is BF16.
 //
 // Written for readability, not speed. All products are accumulated in int64
 // (group dot products) and double (scaled sums), in ascending group order.

@@ -277,6 +277,13 @@ __device__ __forceinline__ void cluster_sync_startup() {
 __device__ __forceinline__ void cluster_arrive_release() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
+// Arrive without release semantics: for a rendezvous whose only purpose is that
+// peers' barriers exist, when their initialization was already published with
+// fence.mbarrier_init.release.cluster (fence_barrier_init) and no other data is read
+// across the cluster. Much cheaper than the release form.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

@@ -327,7 +327,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane < kMaxGroups) {
       mbar_init(&xready[lane], kQ ? 10 : 2);
       mbar_init(&rfull[lane], 1);
-      mbar_init(&lfull[lane], 1);
       mbar_init(&h_full[lane], 1);
       mbar_init(&res_full[lane], 1);
     }
@@ -358,10 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // issues group gi's tiles.
     if (lane < ng) {
       const int gi = lane;
-      if (T::lr) {
-        mbar_arrive_expect_tx(&lfull[gi], 8192);
-        tma_load_2d(ltiles + gi * 8192, &tm_l1q, &lfull[gi], (g0 + gi) * 64, 0);
-      }
       if (T::res) {
         mbar_arrive_expect_tx(&rfull[gi], 8192);
         tma_load_2d(rtiles + gi * 8192, &tm_rq, &rfull[gi], (g0 + gi) * 64, n0);
@@ -374,6 +369,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  if (warp == 2) {
+    // The L1 tiles are requested by warp 2 (idle here), in parallel with warp 0's R tiles:
+    // a warp issues its lanes' TMA requests one after another.
+    if (lane < kMaxGroups) mbar_init(&lfull[lane], 1);
+    fence_barrier_init();
+    __syncwarp();
+    if (T::lr && lane < ng) {
+      mbar_arrive_expect_tx(&lfull[lane], 8192);
+      tma_load_2d(ltiles + lane * 8192, &tm_l1q, &lfull[lane], (g0 + lane) * 64, 0);
+    }
+  }
   if (warp == 1) {
     tmem_alloc(tmem_holder, kTmemCols);
     tmem_relinquish();
@@ -382,8 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   // Cluster rendezvous, split: every thread arrives here, after this CTA's barriers
   // are initialized; only the exchange warps (12-19), the ones that store into peers'
-  // shared memory, wait for the peers' arrivals, just before their first push.
-  cluster_arrive_release();
+  // shared memory, wait for the peers' arrivals, just before their first push. The
+  // arrive is relaxed: the initializations were published by fence.mbarrier_init
+  // (release, cluster scope) in warps 0 and 2, and peers only write into this CTA.
+  cluster_arrive_relaxed();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 

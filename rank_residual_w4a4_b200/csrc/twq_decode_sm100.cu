@@ -9,12 +9,11 @@
 //   * split K: a cluster of KS CTAs shares one column tile; CTA k of the cluster
 //     reduces over its own m/KS slice of the groups, so 4 x (n/128) CTAs stream
 //     the weights at once;
-//   * R codes: every group tile of the CTA is requested by TMA at once (64-byte
-//     swizzle); warps unpack them in registers and write the int8 A operand
-//     straight into tensor memory (tcgen05.st), so shared memory only carries
-//     the packed bytes once;
-//   * L1 codes (mostly L2-resident after the first cluster) are loaded with
-//     plain loads into tensor memory the same way;
+//   * R and L1 codes: every group tile of the CTA is requested by TMA at once
+//     (64-byte swizzle; R tiles by warp 0, L1 tiles by warp 2, in parallel);
+//     warps unpack them in registers and write the int8 A operand straight into
+//     tensor memory (tcgen05.st), so shared memory only carries the packed bytes
+//     once;
 //   * stage 1 gives each CTA a partial H (its groups) for all r; the partials
 //     are pushed over distributed shared memory to the CTA that owns each
 //     16-column unit of r, which sums them in a fixed order, rounds to BF16 and
@@ -22,6 +21,10 @@
 //   * Y partials (residual over the CTA's groups + stage 2 over its r units)
 //     are pushed to the CTA that owns each column slice, summed in a fixed
 //     order, rounded to BF16 and stored once.
+// Variants: the activation quantizer inside the kernel (BF16 X in, kQ), and
+// W4A8 (int8 activation codes, q_max = 127, kA8). The kernel signals programmatic
+// launch completion at entry; every role passes griddepcontrol.wait before it
+// depends on X, which the preceding kernel may produce.
 // Cross-CTA data moves only as st.async pushes into the receiving CTA's shared
 // memory, each completing bytes on the receiver's mbarrier (which registered
 // the exact byte count it expects before the cluster rendezvous). A CTA never

@@ -21,11 +21,19 @@
  *   epilogue Y = bf16_rne(Y_res + Y_lr), one store (§4.3: a single epilogue
  *            merges both components).
  *
- * Memory: every pointer is a DEVICE pointer owned by the caller; the library
- * never allocates, frees or synchronizes (except twq_device_status and the
- * offline twq_fold_transforms). Every
- * call is asynchronous on `stream`; inputs must stay live until the stream
- * reaches the call. All base pointers must be 16-byte aligned.
+ * Variants (declared below): the layer with the activation quantizer inside it
+ * (twq_fused_linear_x, decode batches), from host memory to host memory
+ * (twq_fused_linear_x_host), with 8-bit activations (W4A8, §5.1:
+ * twq_quantize_act_a8 / twq_fused_linear_a8 / twq_fused_linear_x_a8), with the
+ * pages' INT4 stage 2 (twq_pack_l2_int4 / twq_fused_linear_s2q), and the offline
+ * fold of the learned transforms (twq_fold_transforms).
+ *
+ * Memory: every pointer is a DEVICE pointer owned by the caller (except the
+ * x_host / y_host buffers of twq_fused_linear_x_host); the library never
+ * allocates, frees or synchronizes (except twq_device_status and the offline
+ * twq_fold_transforms). Every call is asynchronous on `stream`; inputs must stay
+ * live until the stream reaches the call. All base pointers must be 16-byte
+ * aligned.
  *
  * Errors: arguments are validated on the host before anything is launched; a
  * failing check returns a status and launches nothing. A launch failure is

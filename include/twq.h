@@ -74,7 +74,7 @@ typedef struct CUstream_st* twq_stream_t;
 typedef enum {
   TWQ_OK = 0,
   TWQ_ERR_INVALID_ARG = 1,     /* null pointer, bad shape or size */
-  TWQ_ERR_UNSUPPORTED = 2,     /* valid but outside this build's limits (e.g. r > 256) */
+  TWQ_ERR_UNSUPPORTED = 2,     /* valid but outside the library's limits (e.g. r > 256) */
   TWQ_ERR_MISALIGNED = 3,      /* a pointer or stride breaks the 16-byte rule */
   TWQ_ERR_CUDA = 4,            /* a CUDA runtime/driver call or launch failed */
   TWQ_ERR_NOT_IMPLEMENTED = 5,

@@ -20,7 +20,7 @@
 // * Kernel dataflow, §4.3: one activation quantization reused by the residual
 //   GEMM and the first low-rank GEMM; the first stage's result H is
 //   converted and fed to the second stage; a single epilogue adds both parts.
-//   In this build the second stage takes H rounded to BF16 and L2 in BF16
+//   Here the second stage takes H rounded to BF16 and L2 in BF16
 //   (the page's on-the-fly INT4 requantization is composed from these functions
 //   in oracle.layer_s2q), and Y is BF16.
 //

@@ -250,6 +250,11 @@ __device__ __forceinline__ void st_async_peer_v4u(uint32_t raddr, uint4 v, uint3
       "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(rbar)
       : "memory");
 }
+__device__ __forceinline__ void st_async_peer_u32(uint32_t raddr, uint32_t v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(raddr),
+               "r"(v), "r"(rbar)
+               : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_peer(uint32_t raddr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(raddr)
                : "memory");

@@ -192,7 +192,9 @@ twq_status twq_fused_linear_s2q(const uint8_t* xq, const float* sx, int64_t b, c
   twq::GemmCall c{twq::kModeFusedS2Q, xq, sx, b, w, y, nullptr};
   c.l2q = l2q;
   c.sl2q = sl2q;
-  return from_cuda(twq::launch_gemm(c, reinterpret_cast<cudaStream_t>(stream), nullptr));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (twq::decode_eligible(c)) return from_cuda(twq::launch_decode(c, st));
+  return from_cuda(twq::launch_gemm(c, st, nullptr));
 }
 
 // Validates a twq_fused_linear_x call (b >= 1) and fills the decode launch.

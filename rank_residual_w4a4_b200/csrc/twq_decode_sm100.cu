@@ -60,7 +60,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 enum DecodeSite : int {
   kDSiteX = 21, kDSiteR = 22, kDSiteL1 = 23, kDSiteAl = 24, kDSiteH = 25, kDSiteRes = 26,
   kDSiteAr = 27, kDSiteHReady = 28, kDSiteHb = 29, kDSiteL2 = 30, kDSiteLr = 31,
-  kDSiteYReady = 32, kDSiteFinal = 33,
+  kDSiteYReady = 32, kDSiteFinal = 33, kDSiteHq = 34, kDSiteHmax = 35,
 };
 
 template <int kMode>
@@ -76,6 +76,8 @@ struct DecodeArgs {
   uint16_t* y;
   int64_t b;
   int m, n, r, G;
+  const uint8_t* l2q;  // INT4 stage 2: 4-bit L2 codes, n x r/2 (column j contiguous along r)
+  const float* sl2q;   // INT4 stage 2: their scales, (r/128) x n
 };
 
 struct DLayout {
@@ -91,7 +93,11 @@ struct DLayout {
   static constexpr int kHredBytes = 128 * kNT * 4;             // [src][c][t], KS * slice <= 128
   static constexpr int kOffYred = kOffHred + kHredBytes;
   static constexpr int kYredBytes = 128 * kNT * 4;             // [src][j][t], KS * cols = 128
-  static constexpr int kOffBar = kOffYred + kYredBytes;
+  // INT4 stage 2: per-token maxima of |bf16(H)| from every CTA, s_H, this CTA's maxima
+  static constexpr int kOffHmx = kOffYred + kYredBytes;        // [src][token] fp32
+  static constexpr int kOffShq = kOffHmx + 8 * kNT * 4;         // [token] fp32
+  static constexpr int kOffHloc = kOffShq + kNT * 4;            // [token] fp32 bits (atomicMax)
+  static constexpr int kOffBar = kOffHloc + kNT * 4;
   static constexpr int kNumBars = 64;
   static constexpr int kBytes = kOffBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -257,7 +263,8 @@ __device__ __forceinline__ void unit_range(int U, int KS, int k, int& u0, int& u
 }
 
 // kA8: W4A8, the activation codes are int8 (q_max = 127), one per byte.
-template <int kMode, int KS, bool kQ, bool kA8>
+// kS2Q: the INT4 stage 2 (H requantized on chip, 4-bit L2 codes), r = 128.
+template <int kMode, int KS, bool kQ, bool kA8, bool kS2Q>
 __global__ void __launch_bounds__(kThreads, 1)
     twq_decode_kernel(const __grid_constant__ CUtensorMap tm_rq,
                       const __grid_constant__ CUtensorMap tm_l1q,
@@ -297,8 +304,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* lr_full = hb_ready + 1;
   uint64_t* h_ready = lr_full + 1;
   uint64_t* y_ready = h_ready + 1;
-  uint64_t* mma_done = y_ready + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
+  uint64_t* mma_done = y_ready + 1;           // [2]
+  uint64_t* hmax_ready = mma_done + 2;        // INT4 stage 2: every CTA's per-token maxima
+  uint64_t* hq4 = mma_done + 3;               // INT4 stage 2: the 4 H-owner warps' maxima
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 4);
+  float* hmx = reinterpret_cast<float*>(smem + L::kOffHmx);
+  float* shq = reinterpret_cast<float*>(smem + L::kOffShq);
+  int* hloc = reinterpret_cast<int*>(smem + L::kOffHloc);
   volatile int* abort_flag = &s_abort;
 
   // The next kernel on the stream may be scheduled now: its prologue and weight
@@ -351,7 +363,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(y_ready, KS * kColsPerOwner * kNT * 4);
       mbar_init(mma_done, 1);
       mbar_init(mma_done + 1, 1);
+      if (kS2Q) {  // every CTA sends its 16 per-token maxima to every CTA of the cluster
+        mbar_init(hmax_ready, 1);
+        mbar_arrive_expect_tx(hmax_ready, KS * kNT * 4);
+        mbar_init(hq4, 4);
+      }
       s_abort = 0;
+    }
+    if (kS2Q) {
+      if (lane < kNT) hloc[lane] = 0;
+      // the stage-2 B tile (H's codes) is zero beyond the CTA's slice of r (K padding)
+      for (int e = lane; e < 2048 / 16; e += 32)
+        reinterpret_cast<uint4*>(hbs)[e] = make_uint4(0, 0, 0, 0);
     }
     fence_barrier_init();
     __syncwarp();
@@ -366,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (lane == 31) {
-      if (T::lr && my_units > 0) {
+      if (T::lr && my_units > 0 && !kS2Q) {
         mbar_arrive_expect_tx(l2full, 16384);
         tma_load_2d(l2s, &tm_l2t, l2full, u0 * 16, n0);
       }
@@ -457,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (T::lr) d_wait<false>(&lfull[gi], 0, &never, kDSiteFinal);
         if (T::res) d_wait<false>(&rfull[gi], 0, &never, kDSiteFinal);
       }
-      if (T::lr && my_units > 0) d_wait<false>(l2full, 0, &never, kDSiteFinal);
+      if (T::lr && my_units > 0 && !kS2Q) d_wait<false>(l2full, 0, &never, kDSiteFinal);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -481,7 +504,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&h_full[gi]);
         }
       }
-      if (T::lr && my_units > 0 && ok) {
+      if (kS2Q && T::lr && my_units > 0 && ok) {
+        // INT4 stage 2: A = this CTA's 4-bit L2 codes (128 columns x its slice of r, int8
+        // 16q), B = the codes of H for the slice, K = the slice padded to 32
+        ok = d_wait<true>(hb_ready, 0, abort_flag, kDSiteHb);
+        if (ok) {
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(smem_u32(l2s));
+          const uint64_t db = smem_desc_sw128(smem_u32(hbs));
+          for (int k = 0; k < (my_units + 1) / 2; ++k)
+            mma_i8(tmem_base + kColDlr, da + 2 * k, db + 2 * k, idesc, k > 0);
+          mma_commit(lr_full);
+        }
+      } else if (T::lr && my_units > 0 && ok) {
         ok = d_wait<true>(hb_ready, 0, abort_flag, kDSiteHb) &&
              d_wait<false>(l2full, 0, abort_flag, kDSiteL2);
         if (ok) {
@@ -569,6 +604,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------- stage-1 drain, H exchange, BF16 H for stage 2 (warps 12-15)
     cluster_wait_acquire();  // peers' barriers are initialized before the first push
     pdl_wait();
+    // INT4 stage 2: thread tid holds the 4-bit L2 codes of output column n0 + tid for this
+    // CTA's units of r (8 bytes, 16 codes, per unit), loaded early
+    uint2 l2w[4] = {};
+    if (kS2Q && T::lr)
+      for (int u = 0; u < my_units && u < 4; ++u)
+        l2w[u] = __ldg(reinterpret_cast<const uint2*>(
+            args.l2q + static_cast<int64_t>(n0 + threadIdx.x - 384) * (args.r / 2) + (u0 + u) * 8));
     if (T::lr) {
       const int q = warp & 3;
       const int c = q * 32 + lane;  // index into r
@@ -624,7 +666,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       // into it when it exits); the wait ignores the abort flag for the same reason.
       int keep_waiting = 0;
       const bool got = my_units > 0 ? d_wait<true>(h_ready, 0, &keep_waiting, kDSiteHReady) : true;
-      if (ok && got && my_units > 0) {
+      if constexpr (kS2Q) {
+        // INT4 stage 2 (r = 128): Eq. (1) on bf16(H) per token over all of r. The CTAs
+        // own slices of r, so each sends its per-token maxima to every CTA; all of them
+        // then compute the same scale. Every step runs even after a local failure, so
+        // the exchange stays complete and peers are not left waiting.
+        const int tid = threadIdx.x - 384;
+        const int slice = my_units * 16;  // <= 64
+        const int t = tid & (kNT - 1);    // element e = tid + 128 i has token e % 16 = t
+        float hv[8];
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = tid + 128 * i;
+          hv[i] = 0.0f;
+          if (e < slice * kNT) {
+            const int cl = e / kNT;
+            float h = 0.0f;
+            for (int k = 0; k < KS; ++k) h += hred[(k * kHSlice + cl) * kNT + t];
+            hv[i] = __bfloat162float(__float2bfloat16_rn(h));  // H rounded to BF16 first
+            mx = fmaxf(mx, fabsf(hv[i]));
+          }
+        }
+        if (ok && got) atomicMax(hloc + t, __float_as_int(mx));  // non-negative: int order
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hq4);
+        int keep = 0;
+        d_wait<false>(hq4, 0, &keep, kDSiteHq);
+        if (tid < kNT)
+          for (int k = 0; k < KS; ++k)
+            st_async_peer_u32(map_peer(smem_u32(hmx + ks * kNT + tid), k),
+                              static_cast<uint32_t>(hloc[tid]), map_peer(smem_u32(hmax_ready), k));
+        const bool gotm = d_wait<true>(hmax_ready, 0, &keep, kDSiteHmax);
+        float a = 0.0f;
+        for (int k = 0; k < KS; ++k) a = fmaxf(a, hmx[k * kNT + t]);
+        const Eq1Scale sh = eq1_scale<7>(a);
+        if (tid < kNT) shq[tid] = sh.s;
+        // codes of this thread's elements into the B tile (16 rows, SW128), as 16*q bytes in
+        // the 4-bit operand order: even elements of each 16-element chunk first
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = tid + 128 * i;
+          if (e < slice * kNT) {
+            const int cl = e / kNT, w = cl & 15;
+            uint32_t code = 0;
+            if (sh.s != 0.0f) {
+              const float f1[1] = {hv[i]};
+              uint32_t nb[1];
+              eq1_nibbles(f1, sh, nb);
+              code = nb[0] << 4;
+            }
+            const int pos = (w & 8) + ((w & 1) ? 4 : 0) + ((w & 7) >> 1);
+            hbs[d_sw128(t, cl >> 4) + pos] = static_cast<uint8_t>(code);
+          }
+        }
+        // the A tile: 128 output columns x the slice of r, int8 16q (K padded to 32)
+        {
+          const int j = tid;
+          for (int u = 0; u < 4; ++u) {
+            if (u < ((my_units + 1) / 2) * 2) {
+              uint32_t o[4] = {0, 0, 0, 0};
+              if (u < my_units) unpack8(l2w[u].x, l2w[u].y, o);
+              *reinterpret_cast<uint4*>(l2s + d_sw128(j, u)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        }
+        (void)gotm;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hb_ready);
+      } else if (ok && got && my_units > 0) {
         const int tid = threadIdx.x - 384;
         const int slice = my_units * 16;
         for (int e = tid; e < slice * kNT; e += 128) {
@@ -674,13 +785,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int t = 0; t < kNT; ++t) part[t] = acc[t] * kDq;
     if (T::lr && my_units > 0 && ok) {
+      // INT4 stage 2: s_V of column j for the group of r that holds this CTA's slice
+      const float sv = kS2Q ? __ldg(args.sl2q + static_cast<int64_t>(u0 * 16 / 128) * args.n + n0 + j)
+                            : 0.0f;
       if ((ok = d_wait<false>(lr_full, 0, abort_flag, kDSiteLr))) {
         tc_fence_after();
         uint32_t v[16];
         tmem_ld16(tmem_base + lane_addr + kColDlr, v);
         tmem_wait_ld();
+        if constexpr (kS2Q) {
+          // int32 = 256 x the codes' dot product over the slice; s_H from the H-owner warps,
+          // complete once hb_ready completed (the MMA waited for it)
+          ok = d_wait<false>(hb_ready, 0, abort_flag, kDSiteHb);
 #pragma unroll
-        for (int t = 0; t < kNT; ++t) part[t] += __uint_as_float(v[t]);
+          for (int t = 0; t < kNT; ++t)
+            part[t] += static_cast<float>(static_cast<int32_t>(v[t])) * sv * shq[t] * 0.00390625f;
+        } else {
+#pragma unroll
+          for (int t = 0; t < kNT; ++t) part[t] += __uint_as_float(v[t]);
+        }
       }
     }
     tc_fence_before();
@@ -809,7 +932,7 @@ bool d_encode_raw(CUtensorMap* map, CUtensorMapDataType dt, const void* base, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int kMode, int KS, bool kQ, bool kA8>
+template <int kMode, int KS, bool kQ, bool kA8, bool kS2Q = false>
 cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
   const twq_weights* w = c.w;
   DecodeArgs a{};
@@ -836,11 +959,16 @@ cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
   if (DTraits<kMode>::lr)
     ok = ok && d_encode(&m_l1q, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->l1q, kb, a.r, kb, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_64B);
-  if (DTraits<kMode>::lr)
+  if (DTraits<kMode>::lr && !kS2Q)
     ok = ok && d_encode(&m_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2t, a.r, a.n,
                         static_cast<uint64_t>(a.r) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (kS2Q) {
+    a.l2q = c.l2q;
+    a.sl2q = c.sl2q;
+    ok = ok && c.l2q && c.sl2q;
+  }
   if (!ok) return cudaErrorInvalidValue;
-  auto kern = twq_decode_kernel<kMode, KS, kQ, kA8>;
+  auto kern = twq_decode_kernel<kMode, KS, kQ, kA8, kS2Q>;
   // The shared-memory opt-in is a driver call: once per instantiation and device.
   static std::atomic<uint64_t> smem_set{0};
   int dev = 0;
@@ -878,6 +1006,8 @@ cudaError_t launch_decode_mode(const GemmCall& c, cudaStream_t st) {
 
 bool decode_eligible(const GemmCall& c) {
   const twq_weights* w = c.w;
+  if (c.mode == kModeFusedS2Q) return !c.x && !c.a8 && c.b >= 1 && c.b <= kNT && w->r == 128 &&
+                                      w->m / 128 <= 8 * kMaxGroups && w->n % 128 == 0;
   if (c.mode != kModeFused && c.mode != kModeW4A4 && c.mode != kModeLowRank) return false;
   if (c.a8 && c.mode == kModeLowRank) return false;
   if (c.b < 1 || c.b > kNT) return false;
@@ -895,6 +1025,9 @@ cudaError_t launch_decode(const GemmCall& c, cudaStream_t st) {
                     : launch_decode_mode<MODE, 4, true, A8>(c, st);                       \
   return ks8 ? launch_decode_mode<MODE, 8, false, A8>(c, st)                              \
              : launch_decode_mode<MODE, 4, false, A8>(c, st);
+  if (c.mode == kModeFusedS2Q)  // the INT4 stage 2 (codes in, r = 128)
+    return ks8 ? launch_decode_mode<kModeFused, 8, false, false, true>(c, st)
+               : launch_decode_mode<kModeFused, 4, false, false, true>(c, st);
   if (c.a8) {  // W4A8: the full layer and the residual alone
     switch (c.mode) {
       case kModeFused: { TWQ_DECODE_CASE(kModeFused, true) }

@@ -113,3 +113,28 @@ def test_s2q_differs_from_bf16_stage2_by_the_requantization_only(twq, device):
              + 2 * bf16_ulp(synth.bf16_to_f32(yb)) + 1e-6)
     assert (d <= bound).all()
     _status_clean(twq)
+
+
+DECODE_SHAPES = [  # b <= 16, r = 128: the split-K decode kernel. Clusters of 4 (two 16-wide
+    # units of r per CTA) and of 8 (one unit, K padded to 32), uneven group splits
+    (1, 4096, 512, 128), (7, 4096, 256, 128), (16, 8192, 256, 128), (16, 1024, 384, 128),
+    (5, 640, 128, 128),
+]
+
+
+@pytest.mark.parametrize("b,m,n,r", DECODE_SHAPES)
+def test_s2q_decode_matches_oracle(twq, device, b, m, n, r):
+    x, R, L1, L2 = _operands(b, m, n, r, seed=24)
+    y, _, _ = _run(twq, device, x, R, L1, L2)
+    ref = oracle.layer_s2q(x, R, L1, L2, want=("y", "sh"))
+    _assert_s2q_close(y, ref, L2, "decode %s" % ((b, m, n, r),))
+    _status_clean(twq)
+
+
+def test_s2q_decode_workload(twq, device):
+    wl = synth.WORKLOADS["decode"]
+    x = synth.make_x(wl, b=16, seed=7)
+    R, L1, L2 = synth.make_weights(wl, seed=7)
+    y, _, _ = _run(twq, device, x, R, L1, L2)
+    _assert_s2q_close(y, oracle.layer_s2q(x, R, L1, L2, want=("y", "sh")), L2, "decode16")
+    _status_clean(twq)

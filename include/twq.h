@@ -240,10 +240,12 @@ TWQ_API twq_status twq_fused_linear_x_a8(const uint16_t* x, int64_t ldx, int64_t
  *   L2 contiguous along r, nibbles as the codes format above) and sl2q ((r/128) x n
  *   fp32). Offline, with twq_pack_weights; bit-exact.
  * twq_fused_linear_s2q: xq, sx from twq_quantize_act; w from twq_pack_weights (its
- *   l2t is not read); l2q, sl2q from twq_pack_l2_int4; y b x n BF16. One launch of
- *   the tensor-core GEMM kernel for any b (H never leaves the chip; its codes
- *   overwrite it in shared memory and feed r/128 more int8 K groups of the residual
- *   accumulation). Errors as twq_fused_linear; r outside {128, 256} returns
+ *   l2t is not read); l2q, sl2q from twq_pack_l2_int4; y b x n BF16. One launch; H
+ *   never leaves the chip. Decode batches (b <= 16, r == 128, m <= 8192) run the
+ *   split-K decode kernel, whose CTAs exchange per-token maxima of H over the
+ *   cluster; other shapes run the tensor-core GEMM kernel, where H's codes overwrite
+ *   it in shared memory and feed r/128 more int8 K groups of the residual
+ *   accumulation. Errors as twq_fused_linear; r outside {128, 256} returns
  *   TWQ_ERR_UNSUPPORTED (r == 0: TWQ_ERR_INVALID_ARG).
  */
 TWQ_API twq_status twq_pack_l2_int4(const uint16_t* L2, int64_t r, int64_t n, uint8_t* l2q,

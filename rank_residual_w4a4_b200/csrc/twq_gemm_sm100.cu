@@ -311,7 +311,10 @@ __device__ __forceinline__ const uint4* h_piece(const uint8_t* grp, int row, int
   return reinterpret_cast<const uint4*>(grp + (p >> 3) * 16384 + sw128_offset(row, p & 7));
 }
 
-__device__ __noinline__ void requant_h_row(uint8_t* grp, int row, float* s_out) {
+// push: also store the codes and the scale into CTA `peer` of the cluster (the same
+// addresses there), completing bytes on its barrier `peer_bar` (a CTA pair).
+__device__ __noinline__ void requant_h_row(uint8_t* grp, int row, float* s_out, bool push,
+                                           uint32_t peer, uint32_t peer_bar) {
   float a = 0.0f;
 #pragma unroll 4
   for (int p = 0; p < 16; ++p) {
@@ -324,6 +327,7 @@ __device__ __noinline__ void requant_h_row(uint8_t* grp, int row, float* s_out) 
   }
   const Eq1Scale ks = eq1_scale<7>(a);
   *s_out = ks.s;
+  if (push) st_async_peer_u32(map_peer(smem_u32(s_out), peer), __float_as_uint(ks.s), peer_bar);
 #pragma unroll 1
   for (int c = 0; c < 8; ++c) {
     uint4 o = make_uint4(0, 0, 0, 0);
@@ -341,6 +345,7 @@ __device__ __noinline__ void requant_h_row(uint8_t* grp, int row, float* s_out) 
       o = pack_codes16(nb);
     }
     *reinterpret_cast<uint4*>(grp + sw128_offset(row, c)) = o;
+    if (push) st_async_peer_v4u(map_peer(smem_u32(grp + sw128_offset(row, c)), peer), o, peer_bar);
   }
 }
 
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(hb_ready, T::h_global ? 1 : 8);
     mbar_init(hb_free, 1);
     mbar_init(mma_done, 1);
-    mbar_init(peer_free, 1);
+    mbar_init(peer_free, 8);  // each of the peer's 8 drain warps
     mbar_init(hq, 8);
     s_abort = 0;
     fence_barrier_init();
@@ -638,7 +643,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // drain warps over the first 16 KB of H's BF16 columns [128 g2, 128 g2 + 128)),
           // B = the unpacked 4-bit L2 codes
           if (ti.need_h) {
-            if (!(ok = wait_fast(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) break;
+            if (kPair) {  // half of the codes came from the peer's st.async stores
+              if (!(ok = wait_bar_cluster(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) break;
+              fence_proxy_async_smem();
+            } else if (!(ok = wait_fast(hb_ready, hb_phase, abort_flag, kSiteMmaHb))) {
+              break;
+            }
             hb_phase ^= 1u;
           }
           const uint32_t idesc = idesc_i8(BN);
@@ -772,9 +782,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             sx1 = (row_ok && g + 2 < G) ? __ldg(sx_row + g + 2) : 0.0f;
             if (!(ok = wait_bar(&acc_full[a.idx], a.phase, abort_flag, kSiteDrainAccFull))) break;
             // The first stage-1 accumulator of a row block implies that every earlier MMA of
-            // this CTA, stage 2 of the previous row block included, has completed: the peer
-            // may now overwrite its slice of our H tile.
-            if (kPair && hc == 0 && g == 0 && dw == 0 && lane == 0)
+            // this CTA, stage 2 of the previous row block included, has completed, and this
+            // warp has finished the previous row block (INT4 stage 2: its reads of the
+            // peer's scales). Once all 8 drain warps say so, the peer may overwrite its
+            // slice of our H tile and its scales.
+            if (kPair && hc == 0 && g == 0 && lane == 0)
               mbar_arrive_peer(map_peer(smem_u32(peer_free), static_cast<uint32_t>(prank ^ 1)));
             tc_fence_after();
             if (!(ok = wait_bar(&sc_full[q.idx], q.phase, abort_flag, kSiteDrainScaleFull))) break;
@@ -814,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               } else {
                 uint8_t* dst = hb + (col >> 6) * 16384 + sw128_offset(row_in, (col & 63) >> 3);
                 *reinterpret_cast<uint4*>(dst) = o;
-                if (kPair) {
+                if (kPair && !T::s2q) {  // INT4 stage 2: the codes are pushed instead
                   const uint32_t peer = static_cast<uint32_t>(prank ^ 1);
                   st_async_peer_v4u(map_peer(smem_u32(dst), peer), o,
                                     map_peer(smem_u32(hb_ready), peer));
@@ -835,7 +847,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           // Thread (row, half) takes group `half` of its row: it reads the group's 128 BF16
           // values (16 pieces of 8) into registers, then writes the 16*q codes over the
           // group's first 16 KB (only this thread touches these bytes of this row).
-          if (half < args.r / 128) requant_h_row(hb + half * 32768, row_in, shq + row_in * 2 + half);
+          if (kPair) {
+            // a pair (r = 256): this CTA's H columns are group prank of r; it requantizes
+            // them and stores the codes and scales into both CTAs
+            const uint32_t peer = static_cast<uint32_t>(prank ^ 1);
+            if (half == 0)
+              requant_h_row(hb + prank * 32768, row_in, shq + row_in * 2 + prank, true, peer,
+                            map_peer(smem_u32(hb_ready), peer));
+          } else if (half < args.r / 128) {
+            requant_h_row(hb + half * 32768, row_in, shq + row_in * 2 + half, false, 0, 0);
+          }
         }
         if (!T::out_h) {
           fence_proxy_async_smem();
@@ -843,8 +864,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             // For a pair, one arrival also registers the bytes the peer stores into our
             // H tile (its r/2 columns of the 128 rows, BF16).
-            if (kPair && dw == 0)
-              mbar_arrive_expect_tx(hb_ready, static_cast<uint32_t>(kBM * (args.r / 2) * 2));
+            if (kPair && dw == 0)  // BF16 slice (r/2 columns) or, INT4 stage 2, codes + scales
+              mbar_arrive_expect_tx(hb_ready, T::s2q ? static_cast<uint32_t>(kBM * (128 + 4))
+                                                     : static_cast<uint32_t>(kBM * (args.r / 2) * 2));
             else
               mbar_arrive(hb_ready);
           }
@@ -881,7 +903,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (T::s2q) {
         // INT4 stage 2 as r/128 more groups of the same accumulation: I * s_V[col] * s_H[row]
         if (ti.need_h) {  // the requantized H and its scales are complete
-          if (!(ok = wait_bar(hb_ready, hbq_phase, abort_flag, kSiteDrainHbq))) break;
+          if (!(ok = kPair ? wait_bar_cluster(hb_ready, hbq_phase, abort_flag, kSiteDrainHbq)
+                           : wait_bar(hb_ready, hbq_phase, abort_flag, kSiteDrainHbq)))
+            break;
           hbq_phase ^= 1u;
         }
         for (int g2 = 0; g2 < args.r / 128; ++g2) {
@@ -1075,8 +1099,10 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
   // only where that saves more than the SMs that pairs leave idle (clusters are
   // placed within a GPC): the choice compares the K-group steps of the busiest CTA.
   bool pair = false;
-  if constexpr (T::h && T::s2 && !T::h_global) {
-    if (a.col_tiles % 2 == 0 && a.r % 32 == 0 && a.r > kHChunk && a.r <= 2 * kHChunk) {
+  if constexpr (T::h && (T::s2 || T::s2q) && !T::h_global) {
+    // (INT4 stage 2: each CTA of a pair then owns exactly one group of 128 of r)
+    if (a.col_tiles % 2 == 0 && a.r % 32 == 0 && a.r > kHChunk && a.r <= 2 * kHChunk &&
+        (!T::s2q || a.r == 2 * kHChunk)) {
       const int pairs = resident_pairs<kMode, BN, kA8>();
       const int hc1 = (a.r + kHChunk - 1) / kHChunk;
       const int kc = (a.r + 63) / 64;
@@ -1120,7 +1146,7 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
                          static_cast<uint64_t>(a.r) * 2, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
 
-  if (!pair || !(T::h && T::s2 && !T::h_global)) {
+  if (!pair || !(T::h && (T::s2 || T::s2q) && !T::h_global)) {
     auto kern = twq_gemm_kernel<kMode, BN, false, kA8>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -1129,7 +1155,7 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
     kern<<<grid, kThreads, L::kAlloc, st>>>(m_xq, m_rq, m_l1q, m_l2t, m_h, a);
     return cudaGetLastError();
   }
-  if constexpr (T::h && T::s2 && !T::h_global) {
+  if constexpr (T::h && (T::s2 || T::s2q) && !T::h_global) {
   auto kern = twq_gemm_kernel<kMode, BN, true, kA8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;

@@ -105,7 +105,11 @@ TWQ_API const char* twq_status_string(twq_status s);
  */
 TWQ_API twq_status twq_weights_sizes(int64_t m, int64_t n, int64_t r, size_t bytes_out[5]);
 
-/* Byte sizes of {xq, sx} for b tokens of width m. Host only. */
+/*
+ * Byte sizes of {xq, sx} for b tokens of width m. Host only; TWQ_ERR_INVALID_ARG
+ * on b < 0 or m not a positive multiple of 128, TWQ_ERR_UNSUPPORTED beyond the
+ * quantizer's limits (m > 2^24 or b > 2^30).
+ */
 TWQ_API twq_status twq_act_sizes(int64_t b, int64_t m, size_t bytes_out[2]);
 
 /*

@@ -88,6 +88,7 @@ twq_status twq_weights_sizes(int64_t m, int64_t n, int64_t r, size_t bytes_out[5
 
 twq_status twq_act_sizes(int64_t b, int64_t m, size_t bytes_out[2]) {
   if (!bytes_out || b < 0 || m <= 0 || m % 128) return TWQ_ERR_INVALID_ARG;
+  if (m > (int64_t(1) << 24) || b > (int64_t(1) << 30)) return TWQ_ERR_UNSUPPORTED;
   bytes_out[0] = static_cast<size_t>(b * (m / 2));
   bytes_out[1] = static_cast<size_t>(b * (m / 128) * 4);
   return TWQ_OK;

@@ -61,6 +61,13 @@ def test_weight_sizes_closed_form(lib):
     assert twq.act_sizes(16, 4096) == (16 * 2048, 16 * 32 * 4)
 
 
+@pytest.mark.parametrize("b,m,want", [(-1, 128, 1), (1, 100, 1), (1, 0, 1), (1, (1 << 24) + 128, 2),
+                                      ((1 << 30) + 1, 128, 2)])
+def test_act_sizes_rejects_bad_shapes(lib, b, m, want):
+    arr = (ctypes.c_size_t * 2)()
+    assert lib.twq_act_sizes(b, m, arr) == want
+
+
 @pytest.mark.parametrize("m,n,r,want", [(100, 128, 16, 1), (128, 100, 16, 1), (128, 128, 8, 1),
                                         (128, 128, 272, 2), (0, 128, 0, 1), (128, 128, -16, 1)])
 def test_weight_sizes_rejects_bad_shapes(lib, m, n, r, want):

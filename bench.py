@@ -420,7 +420,8 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4 codes -> int8 MMA (s32 acc) + fp32 scales; bf16 stage 2 and output",
+        "dtype": "int8",
+        "dtype_detail": "int4 codes -> int8 MMA (s32 acc) + fp32 scales; bf16 stage 2 and output",
         "data": "synthetic (seeded generator; no dataset or trained weights)",
         "config": {"workload": "%s: b=%d m=%d n=%d r=%d, group 128" % (name, b, wl.m, wl.n, wl.r),
                    "b": b, "m": wl.m, "n": wl.n, "r": wl.r, "parallelism": "replicas x%d" % world,
@@ -715,7 +716,8 @@ def run_reference(args):
         "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8 codes, int64 / fp64 accumulation (CPU oracle)",
+        "dtype": "f64",
+        "dtype_detail": "int8 codes, int64 group dot products, fp64 sums (CPU oracle)",
         "data": "synthetic (seeded generator; no dataset or trained weights)",
         "config": {"workload": "%s: b=%d m=%d n=%d r=%d, group 128" % (name, b, wl.m, wl.n, wl.r),
                    "b": b, "m": wl.m, "n": wl.n, "r": wl.r, "parallelism": "host threads"},

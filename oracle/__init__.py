@@ -24,13 +24,16 @@ FUSED, W4A4_ONLY, LOWRANK_ONLY = 0, 1, 2
 GROUP = 128
 
 
+# IEEE float semantics: no fast-math, no contraction, SSE2 floats
+CXX = ["g++", "-std=c++17", "-O2", "-fno-fast-math", "-ffp-contract=off", "-msse2",
+       "-mfpmath=sse", "-fPIC", "-shared"]
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle with IEEE float semantics (no fast-math, no contraction)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call(
-            ["g++", "-std=c++17", "-O2", "-fno-fast-math", "-ffp-contract=off", "-msse2",
-             "-mfpmath=sse", "-fPIC", "-shared", "-o", tmp, _SRC])
+        subprocess.check_call(CXX + ["-o", tmp, _SRC])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -40,33 +43,38 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int64
 
 
+def _load(path):
+    """The oracle's C library at `path`, with its argument types declared."""
+    lib = ctypes.CDLL(path)
+    for name, args in {
+        "twq_ref_quant_group_f32": [_P, ctypes.c_int, _P, _P],
+        "twq_ref_quant_group_f32_a8": [_P, ctypes.c_int, _P, _P],
+        "twq_ref_quantize_rows_q": [_P, _I, _I, _I, ctypes.c_int, _P, _P],
+        "twq_ref_quantize_rows": [_P, _I, _I, _I, _P, _P],
+        "twq_ref_quantize_cols": [_P, _I, _I, _P, _P],
+        "twq_ref_pack_nibbles": [_P, _I, _P],
+        "twq_ref_unpack_nibbles": [_P, _I, _P],
+        "twq_ref_quantize_act": [_P, _I, _I, _I, _P, _P],
+        "twq_ref_pack_weights": [_P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P],
+        "twq_ref_linear": [_P, _P, _I, _I, _P, _P, _I, _P, _P, _I, _P, ctypes.c_int, _P, _I,
+                           _P, _P, _P, _P],
+        "twq_ref_dequant_matmul": [_P, _P, _I, _I, _P, _P, _I, _P, _P, _I, _P, ctypes.c_int,
+                                   _P],
+    }.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.twq_ref_f32_to_bf16.argtypes = [ctypes.c_float]
+    lib.twq_ref_f32_to_bf16.restype = ctypes.c_uint16
+    lib.twq_ref_qmax.restype = ctypes.c_int
+    lib.twq_ref_qmax_a8.restype = ctypes.c_int
+    return lib
+
+
 def _get():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        for name, args in {
-            "twq_ref_quant_group_f32": [_P, ctypes.c_int, _P, _P],
-            "twq_ref_quant_group_f32_a8": [_P, ctypes.c_int, _P, _P],
-            "twq_ref_quantize_rows_q": [_P, _I, _I, _I, ctypes.c_int, _P, _P],
-            "twq_ref_quantize_rows": [_P, _I, _I, _I, _P, _P],
-            "twq_ref_quantize_cols": [_P, _I, _I, _P, _P],
-            "twq_ref_pack_nibbles": [_P, _I, _P],
-            "twq_ref_unpack_nibbles": [_P, _I, _P],
-            "twq_ref_quantize_act": [_P, _I, _I, _I, _P, _P],
-            "twq_ref_pack_weights": [_P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P],
-            "twq_ref_linear": [_P, _P, _I, _I, _P, _P, _I, _P, _P, _I, _P, ctypes.c_int, _P, _I,
-                               _P, _P, _P, _P],
-            "twq_ref_dequant_matmul": [_P, _P, _I, _I, _P, _P, _I, _P, _P, _I, _P, ctypes.c_int,
-                                       _P],
-        }.items():
-            f = getattr(lib, name)
-            f.argtypes = args
-            f.restype = ctypes.c_int
-        lib.twq_ref_f32_to_bf16.argtypes = [ctypes.c_float]
-        lib.twq_ref_f32_to_bf16.restype = ctypes.c_uint16
-        lib.twq_ref_qmax.restype = ctypes.c_int
-        lib.twq_ref_qmax_a8.restype = ctypes.c_int
-        _lib = lib
+        _lib = _load(build())
     return _lib
 
 

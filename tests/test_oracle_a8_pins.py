@@ -106,6 +106,18 @@ def test_w4a8_layer_brute_force(b, m, n, r, mode):
         ql1, sl1 = oracle.quantize_cols(L1)
     else:
         ql1 = sl1 = L2 = None
-    y = oracle.linear(qx, sx, qr, sr, ql1, sl1, L2, mode=mode, want=("y64",))["y64"]
+    out = oracle.linear(qx, sx, qr, sr, ql1, sl1, L2, mode=mode, want=("y64", "hb"))
     ref = oracle.dequant_matmul(qx, sx, qr, sr, ql1, sl1, L2, mode=mode)
-    assert np.abs(y - ref).max() <= 1e-12 * max(np.abs(ref).max(), 1e-30)
+    assert np.abs(out["y64"] - ref).max() <= 1e-12 * max(np.abs(ref).max(), 1e-30)
+    # and outside the oracle's C code: numpy dequantization, ungrouped fp64 matmuls, stage 2
+    # on the oracle's BF16 H (whose fp64 -> float32 -> BF16 chain numpy re-derives)
+    xd = qx.astype(np.float64) * np.repeat(sx.astype(np.float64), 128, axis=1)
+    rd = np.repeat(sr.astype(np.float64), 128, axis=0) * qr.T.astype(np.float64)
+    ref_np = xd @ rd
+    if r and mode == oracle.FUSED:
+        l1d = np.repeat(sl1.astype(np.float64), 128, axis=0) * ql1.T.astype(np.float64)
+        h = xd @ l1d
+        assert np.flatnonzero(out["hb"] != synth.f32_to_bf16(h.astype(np.float32))).size <= 1
+        ref_np = ref_np + (synth.bf16_to_f32(out["hb"]).astype(np.float64)
+                           @ synth.bf16_to_f32(L2).astype(np.float64))
+    assert np.abs(out["y64"] - ref_np).max() <= 1e-12 * max(np.abs(ref_np).max(), 1e-30)

@@ -188,6 +188,29 @@ def test_brute_force_dequantize_then_matmul(b, m, n, r, mode):
     assert np.abs(y - ref).max() <= 1e-12 * scale
 
 
+@pytest.mark.parametrize("b,m,n,r", [(3, 256, 17, 1), (4, 128, 64, 16), (2, 384, 40, 32)])
+@pytest.mark.parametrize("mode", [oracle.FUSED, oracle.W4A4_ONLY, oracle.LOWRANK_ONLY])
+def test_brute_force_in_numpy(b, m, n, r, mode):
+    """Outside the oracle's C code: dequantize with numpy (s*q per group, Eq. (1)), one
+    ungrouped fp64 matmul per GEMM, and bf16(float32(H)) for stage 2. The oracle's H bits
+    may differ from numpy's only where the two fp64 sums straddle a float32 rounding
+    boundary; Y is then compared on the oracle's own BF16 H."""
+    qx, sx, qr, sr, ql1, sl1, L2 = _tiny_operands(b, m, n, r, seed=31)
+    out = oracle.linear(qx, sx, qr, sr, ql1, sl1, L2, mode=mode, want=("y64", "hb"))
+    xd = qx.astype(np.float64) * np.repeat(sx.astype(np.float64), 128, axis=1)    # b x m
+    rd = np.repeat(sr.astype(np.float64), 128, axis=0) * qr.T.astype(np.float64)   # m x n
+    l1d = np.repeat(sl1.astype(np.float64), 128, axis=0) * ql1.T.astype(np.float64)  # m x r
+    h = xd @ l1d
+    hb_np = synth.f32_to_bf16(h.astype(np.float32))
+    mism = np.flatnonzero(out["hb"] != hb_np) if mode != oracle.W4A4_ONLY else np.array([])
+    assert mism.size <= max(1, h.size // 500)
+    hb = synth.bf16_to_f32(out["hb"]).astype(np.float64) if mode != oracle.W4A4_ONLY else 0.0
+    yres = xd @ rd
+    ylr = hb @ synth.bf16_to_f32(L2).astype(np.float64) if mode != oracle.W4A4_ONLY else 0.0
+    ref = {oracle.FUSED: yres + ylr, oracle.W4A4_ONLY: yres, oracle.LOWRANK_ONLY: ylr}[mode]
+    assert np.abs(out["y64"] - ref).max() <= 1e-12 * max(np.abs(ref).max(), 1e-30)
+
+
 def test_stage2_is_a_plain_matmul_of_bf16_h():
     """Y_lr = bf16(H) @ L2: checked with numpy's matmul on the oracle's own H bits, and
     H itself against the fp64 dequantized product (a second, ungrouped route)."""

@@ -194,3 +194,69 @@ def test_a_planted_mistake_fails_a_pin(name, monkeypatch):
     monkeypatch.setattr(oracle, "_lib", _mutant_lib(name))
     failed = _failures()
     assert failed, "mutant %s passed every check" % name
+
+
+# ------------------------------------------- mistakes in the Python-side oracle
+# The INT4 stage 2 (layer_s2q) and the transform fold (fold_transforms) are written
+# in oracle/__init__.py. A mistake is planted in a copy of that module's source,
+# which runs in place of the oracle under the pins of test_oracle_s2q_pins.py and
+# test_fold_oracle.py (numpy re-derivations, closed forms and identities).
+
+PY_MUTANTS = {
+    "s2q_residual_dropped": ("    total = res + ylr\n", "    total = ylr\n"),
+    "s2q_sign": ("    total = res + ylr\n", "    total = res - ylr\n"),
+    "s2q_h_codes_8bit": ("qh, sh = quantize_rows(hb)", "qh, sh = quantize_rows(hb, a8=True)"),
+    "s2q_v_scales_dropped": ("ylr = linear(qh, sh, qv, sv,", "ylr = linear(qh, sh, qv, np.ones_like(sv),"),
+    "s2q_h_scales_dropped": ("ylr = linear(qh, sh, qv, sv,", "ylr = linear(qh, np.ones_like(sh), qv, sv,"),
+    "fold_q_not_transposed": ("l1 = q.T @ (u @ g)", "l1 = q @ (u @ g)"),
+    "fold_g_inverse_on_u": ("l1 = q.T @ (u @ g)", "l1 = q.T @ (u @ np.linalg.inv(g))"),
+    "fold_g_not_inverted": ("l2 = np.linalg.inv(g) @ v", "l2 = g @ v"),
+    "fold_r_not_transposed": ("rr = q.T @ r", "rr = q @ r"),
+}
+
+
+def _python_pins():
+    import test_fold_oracle as fold
+    import test_oracle_s2q_pins as s2q
+    return [
+        ("s2q codes and brute force r=128", s2q, lambda: s2q.test_codes_and_brute_force(3, 256, 128, 128)),
+        ("s2q codes and brute force r=256", s2q, lambda: s2q.test_codes_and_brute_force(4, 384, 256, 256)),
+        ("s2q exact V", s2q, s2q.test_exact_v_reduces_to_dequantized_h_times_l2),
+        ("s2q two groups of r", s2q, s2q.test_two_groups_of_r_have_their_own_scales),
+        ("fold identities", fold, fold.test_identity_transforms_leave_the_factors_unchanged),
+        ("fold signed permutations", fold, fold.test_signed_permutations_are_exact),
+        ("fold preserves the layer", fold, fold.test_fold_preserves_the_layer_output),
+    ]
+
+
+def _python_failures(module, monkeypatch):
+    failed = []
+    for name, test_module, run in _python_pins():
+        monkeypatch.setattr(test_module, "oracle", module)
+        try:
+            run()
+        except (AssertionError, ValueError):
+            failed.append(name)
+    return failed
+
+
+def _mutant_module(name):
+    import types
+    old, new = PY_MUTANTS[name]
+    path = oracle.__file__
+    with open(path) as fh:
+        src = fh.read()
+    assert src.count(old) == 1, "the planted line is no longer in the oracle: %r" % old
+    mod = types.ModuleType("oracle_mutant_" + name)
+    mod.__file__ = path
+    exec(compile(src.replace(old, new), path, "exec"), mod.__dict__)
+    return mod
+
+
+def test_the_python_oracle_passes_its_pins(monkeypatch):
+    assert _python_failures(oracle, monkeypatch) == []
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_a_planted_python_mistake_fails_a_pin(name, monkeypatch):
+    assert _python_failures(_mutant_module(name), monkeypatch), "mutant %s passed every pin" % name

@@ -52,8 +52,11 @@ WORKLOADS = {
     "large": ("large", 8192),
     "tiny": ("tiny", 16),
 }
-DEFAULT_WORKLOAD = "decode16"
-SWEEP = ["decode1", "decode4", "gateup", "down", "large"]
+# The headline line is the largest single-GPU workload (the Qwen3-32B-like MLP layer);
+# the other workloads are reported in the sweep.
+DEFAULT_WORKLOAD = "large"
+SWEEP = ["decode16", "decode1", "decode4", "gateup", "down"]
+MIN_TIMED_LAUNCHES = 200  # kernel-level timings: at least this many launches, median of replays
 
 
 # ------------------------------------------------------------------ arithmetic
@@ -312,23 +315,63 @@ def time_graph(g, world, device):
     return s.elapsed_time(e) / 1e3  # seconds
 
 
-def kernel_only_time(prob, fn, steps, reps=1):
-    """Average seconds per launch of `fn(i)` captured back-to-back in a graph."""
+def launch_plan(prob):
+    """Launches per graph and graph replays for a kernel-level timing: a graph of
+    back-to-back launches covering the weight rotation (at least 20 launches, a
+    multiple of the copies), replayed until at least MIN_TIMED_LAUNCHES launches
+    have been timed (at least 5 replays)."""
+    per = max(prob.copies, 20 if prob.b > 16 else MIN_TIMED_LAUNCHES)
+    per = -(-per // prob.copies) * prob.copies
+    return per, max(5, -(-MIN_TIMED_LAUNCHES // per))
+
+
+def kernel_only_time(prob, fn):
+    """Median over graph replays of the seconds per launch of `fn(i)`, the launches
+    captured back-to-back in one graph (no events between launches, which would
+    serialize programmatically launched kernels)."""
     import torch
-    g = capture(fn, steps)
+    per, replays = launch_plan(prob)
+    g = capture(fn, per)
     g.replay()
     torch.cuda.synchronize()
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(reps):
+    times = []
+    for _ in range(replays):
+        s.record()
         g.replay()
-    e.record()
+        e.record()
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e) / 1e3 / per)
+    del g
+    return float(np.median(times))
+
+
+def measure_int8_peak(device, n=8192, reps=10):
+    """Dense INT8 tensor throughput of the box, measured like the BF16 entry of the
+    measured peaks: torch._int_mm (cuBLASLt, int8 x int8 -> int32) on n x n x n, best
+    of `reps` CUDA-event timings, in TOPS (2 n^3 ops). A roofline denominator only;
+    nothing on the layer's path uses it."""
+    import torch
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device)
+    torch._int_mm(a, b)
     torch.cuda.synchronize()
-    return s.elapsed_time(e) / 1e3 / (steps * reps)
+    best = float("inf")
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    for _ in range(reps):
+        s.record()
+        torch._int_mm(a, b)
+        e.record()
+        torch.cuda.synchronize()
+        best = min(best, s.elapsed_time(e) / 1e3)
+    del a, b
+    torch.cuda.empty_cache()
+    return 2.0 * n ** 3 / best / 1e12
 
 
-def roofline_entry(name, t_kernel, peaks, traffic, bf16_x=False):
+def roofline_entry(name, t_kernel, peaks, traffic, bf16_x=False, int8_measured=None):
     wl, b = describe(name)
     hbm, bf16, bf16_sus, src = peaks
     m, n, r = wl.m, wl.n, wl.r
@@ -341,15 +384,35 @@ def roofline_entry(name, t_kernel, peaks, traffic, bf16_x=False):
     ops = int8_ops(b, m, n, r) + bf16_flops(b, n, r)
     ach = ops / t_kernel / 1e12
     peak = bf16 * INT8_PER_BF16
-    return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
-            "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": traffic,
-            "peak_source": "%s bf16 burst x %g (nominal int8/bf16 dense ratio)" % (src, INT8_PER_BF16),
-            "algorithmic_ops": ops}
+    out = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
+           "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": traffic,
+           "peak_source": "%s bf16 burst x %g (nominal int8/bf16 dense ratio)" % (src, INT8_PER_BF16),
+           "algorithmic_ops": ops}
+    if int8_measured:
+        out["int8_peak_measured"] = round(int8_measured, 1)
+        out["frac_of_int8_measured"] = round(ach / int8_measured, 4)
+    return out
+
+
+def sample_rows(b, per_block=1, block=128, seed=0):
+    """Rows for the output check: `per_block` seeded rows from every `block`-row block
+    (every row block of the persistent schedule is looked at), plus the last row."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for r0 in range(0, b, block):
+        hi = min(b, r0 + block)
+        rows.extend(sorted(rng.choice(np.arange(r0, hi), size=min(per_block, hi - r0), replace=False)))
+    rows.append(b - 1)
+    return np.unique(np.array(rows, dtype=np.int64))
 
 
 def run_gpu(args):
     import torch
     world, rank, local = dist_setup()
+    if args.gpus != world:
+        raise SystemExit("bench.py: --gpus %d but %d rank(s) were launched; for N > 1 launch N "
+                         "ranks with python -m torch.distributed.run --nproc-per-node N "
+                         "(one process per GPU)" % (args.gpus, world))
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -361,6 +424,7 @@ def run_gpu(args):
     _build.build()
     twq.load()
     peaks = load_peaks()
+    int8_peak = measure_int8_peak(device)
     name = args.workload
     prob = Problem(name, device)
     K, W = args.steps, args.warmup
@@ -381,27 +445,44 @@ def run_gpu(args):
     t_load0 = time.time()
     # keep the GPU busy for a while so the clock samples see it under load
     t_end = time.time() + args.clock_seconds
+    gw.replay()
+    torch.cuda.synchronize()
     while time.time() < t_end:
         gw.replay()
         torch.cuda.synchronize()
     elapsed = time_graph(gk, world, device)
     t_load1 = time.time()
     elapsed = max_over_ranks(elapsed, world, device)
-    # the layer kernel alone: CUDA events around a graph of K back-to-back launches
-    # on the same stream and weight rotation (no events between launches, which
-    # would serialize them)
+    del gk, gw
+    # the layer kernel alone (and the quantizer alone): CUDA events around graphs of
+    # back-to-back launches on the same stream and weight rotation
     def fused_only(i):
         c = i % prob.copies
         twq.fused_linear(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c])
+
+    def quant_only(i):
+        c = i % prob.copies
+        twq.quantize_act(prob.x[c], prob.xq[c], prob.sx[c])
+
     one = prob.one_launch
-    t_fused = kernel_only_time(prob, prob.step_x if one else fused_only, K)
+    t_fused = kernel_only_time(prob, prob.step_x if one else fused_only)
+    t_quant = None if one else kernel_only_time(prob, quant_only)
     t_two = time_graph(capture(prob.step_two_call, K), world, device) / K if one else None
     t_a8 = time_graph(capture(prob.step_x_a8, K), world, device) / K if one else None
     st = twq.device_status()
     if st != 0:
         raise RuntimeError("device wait timed out at site %d" % st)
 
-    # end to end through the public binding, host buffers, copies inside the timed region
+    # the benched step once more, outside any graph, for the output check below
+    prob.step(0)
+    torch.cuda.synchronize()
+    rows = sample_rows(b)
+    y_rows = prob.y[0][torch.as_tensor(rows, device=device)].view(torch.int16).cpu().numpy().view(np.uint16)
+    yf = y_rows.astype(np.uint32) << 16
+    if not np.isfinite(yf.view(np.float32)).all():
+        raise RuntimeError("non-finite output in the benched step: no number is reported")
+
+    # end to end through the public C ABI, host buffers, copies inside the timed region
     e2e = run_e2e(prob, K, W, world, device)
     clocks.stop()
     clk = clocks.summary(t_load0, t_load1)
@@ -409,6 +490,7 @@ def run_gpu(args):
     tokens = b * world * K
     value = tokens / elapsed
     ops = int8_ops(b, wl.m, wl.n, wl.r) + bf16_flops(b, wl.n, wl.r)
+    per, replays = launch_plan(prob)
     line = {
         "metric": "fused W4A4+low-rank linear: effective TOPS & tokens/s; % of HBM / INT8 roofline",
         "value": round(value, 1),
@@ -427,19 +509,33 @@ def run_gpu(args):
                    "b": b, "m": wl.m, "n": wl.n, "r": wl.r, "parallelism": "replicas x%d" % world,
                    "step": ("twq_fused_linear_x (activation quantizer inside the layer kernel)"
                             if one else "twq_quantize_act + twq_fused_linear"),
-                   "l2": "weights rotate over %d copies (%.0f MB > 2x L2)" % (
-                       prob.copies, prob.copies * weight_bytes(wl.m, wl.n, wl.r) / 1e6),
-                   "launch": "CUDA graph of the K timed steps; the fused kernel is "
-                             "launched with programmatic stream serialization"},
+                   "l2": "inputs larger than L2: weights rotate over %d copies (%.0f MB > 2x L2); "
+                         "X %.0f MB and Y %.0f MB per step" % (
+                             prob.copies, prob.copies * weight_bytes(wl.m, wl.n, wl.r) / 1e6,
+                             2 * b * wl.m / 1e6, 2 * b * wl.n / 1e6),
+                   "launch": "CUDA graph of the K timed steps" + (
+                       "; the layer kernel is launched with programmatic stream serialization"
+                       if one else "")},
         "effective_tops": round(ops * world * K / elapsed / 1e12, 3),
         "fused_kernel_us": round(t_fused * 1e6, 3),
-        "fused_kernel_timing": "events around a graph of K back-to-back layer launches",
+        "fused_kernel_timing": "median over %d replays of a graph of %d back-to-back layer "
+                               "launches (%d launches timed)" % (replays, per, per * replays),
         "roofline": roofline_entry(name, t_fused, peaks,
-                                   profiled_traffic(name + ("_x" if one else "")), bf16_x=one),
+                                   profiled_traffic(name + ("_x" if one else "")), bf16_x=one,
+                                   int8_measured=int8_peak),
+        "int8_peak_tops": round(int8_peak, 1),
+        "int8_peak_how": "torch._int_mm 8192^3 (cuBLASLt), best of 10, CUDA events, this run",
         "e2e": e2e,
         "gpu_launches": (1 if one else 2) * K,
         "clocks": clk,
     }
+    if t_quant is not None:
+        line["quantize_us"] = round(t_quant * 1e6, 3)
+        qb = b * wl.m * 2 + b * wl.m // 2 + 4 * b * (wl.m // 128)
+        line["quantize_roofline"] = {"bound": "hbm", "achieved": round(qb / t_quant / 1e9, 1),
+                                     "peak": peaks[0], "unit": "GB/s",
+                                     "frac": round(qb / t_quant / 1e9 / peaks[0], 4),
+                                     "algorithmic_bytes": qb}
     if one:
         line["two_call_step_us"] = round(t_two * 1e6, 3)
         line["two_call_step"] = "twq_quantize_act + twq_fused_linear, same graph timing"
@@ -447,44 +543,59 @@ def run_gpu(args):
         line["w4a8_step"] = ("twq_fused_linear_x_a8: the same layer with 8-bit activation codes "
                              "(W4A8), same graph timing")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(name, seconds=args.cpu_seconds)
+        cpu = cpu_baseline(name, seconds=args.cpu_seconds, check=(rows, y_rows))
+        line["cpu_baseline"] = cpu
+        if not cpu["output_check"]["ok"]:
+            raise RuntimeError("the benched step's output differs from the oracle on sampled rows "
+                               "(%s): no number is reported" % json.dumps(cpu["output_check"]))
     if rank == 0 and world == 1 and not args.no_sweep:
-        line["sweep"] = sweep(args, device, peaks)
+        line["sweep"] = sweep(args, device, peaks, int8_peak)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del gk, gw
         dist.destroy_process_group()
 
 
 def run_e2e(prob, K, W, world, device):
-    """Same metric through the Python binding with host buffers: per step an H2D copy of
-    X from pinned memory, the layer step of run_gpu, and a D2H copy of Y."""
+    """Same metric through the C ABI with host buffers: per step the H2D copy of X from
+    pinned memory, the layer and the D2H copy of Y are enqueued by C-ABI calls that take
+    host pointers (twq_fused_linear_x_host for decode batches, twq_linear_host otherwise),
+    rotating over four streams with their own device buffers so that one stream's copies
+    overlap another's kernels. Prefill batches are issued in row chunks, one call each."""
     import torch
     from rank_residual_w4a4_b200 import twq
     xh = torch.from_numpy(prob.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-    # Decode steps rotate over four streams, each with its own device and pinned host
-    # buffers, so a step's copies (about 6 us each way for 128 KB) overlap the other
-    # streams' layer kernels; with fewer streams the per-stream chain H2D -> layer ->
-    # D2H sets the pace.
-    streams = [torch.cuda.Stream(device) for _ in range(4)]
-    xds = [torch.empty_like(prob.x[0]) for _ in streams]
-    yds = [torch.empty_like(prob.y[0]) for _ in streams]
-    yhs = [torch.empty((prob.b, prob.n), dtype=torch.bfloat16).pin_memory() for _ in streams]
-    steps = ([twq.DecodeStep(xds[j], yds[j], yhs[j], stream=streams[j]) for j in range(len(streams))]
-             if prob.one_launch else None)
+    nstreams = 4
+    streams = [torch.cuda.Stream(device) for _ in range(nstreams)]
+    if prob.one_launch:
+        xds = [torch.empty_like(prob.x[0]) for _ in streams]
+        yds = [torch.empty_like(prob.y[0]) for _ in streams]
+        yhs = [torch.empty((prob.b, prob.n), dtype=torch.bfloat16).pin_memory() for _ in streams]
+        calls = [twq.DecodeStep(xds[j], yds[j], yhs[j], stream=streams[j]) for j in range(nstreams)]
+        chunks = [(0, prob.b)]
+        path = ("twq_fused_linear_x_host (H2D, the one-launch layer, D2H in one C-ABI call) via "
+                "twq.DecodeStep, eager, four streams in rotation")
+    else:
+        chunk = max(1, min(prob.b, 1024))
+        chunks = [(r0, min(prob.b, r0 + chunk)) for r0 in range(0, prob.b, chunk)]
+        yh = torch.empty((prob.b, prob.n), dtype=torch.bfloat16).pin_memory()
+        # chunk k always runs on stream k % 4, with its own device buffers and its own
+        # rows of the pinned host Y
+        calls = [twq.LinearHostStep(r1 - r0, prob.m, prob.n, device,
+                                    stream=streams[k % nstreams], y_host=yh[r0:r1])
+                 for k, (r0, r1) in enumerate(chunks)]
+        path = ("twq_linear_host (H2D, twq_quantize_act, twq_fused_linear, D2H in one C-ABI call) "
+                "per %d-row chunk via twq.LinearHostStep, eager, four streams in rotation" % chunk)
+    xparts = [xh[r0:r1] for r0, r1 in chunks]
 
     def one(i):
         c = i % prob.copies
         if prob.one_launch:
-            steps[i % len(steps)](xh, prob.weights[c])
+            calls[i % nstreams](xparts[0], prob.weights[c])
         else:
-            xd = xds[0]
-            xd.copy_(xh, non_blocking=True)
-            xq, sx = twq.quantize_act(xd, prob.xq[c], prob.sx[c])
-            y = twq.fused_linear(xq, sx, prob.weights[c], prob.y[c])
-            yhs[0].copy_(y, non_blocking=True)
+            for k, xp in enumerate(xparts):
+                calls[k](xp, prob.weights[c])
 
     for i in range(W):
         one(i)
@@ -500,7 +611,7 @@ def run_e2e(prob, K, W, world, device):
     for i in range(K):
         one(i)
     host_s = time.perf_counter() - h0  # host time to issue the K steps
-    for st in streams:  # ... and e waits for both of them
+    for st in streams:  # ... and e waits for all of them
         cur.wait_stream(st)
     e.record(cur)
     torch.cuda.synchronize()
@@ -509,12 +620,10 @@ def run_e2e(prob, K, W, world, device):
     return {"value": round(prob.b * world * K / t, 1), "unit": "tokens/s",
             "h2d_bytes_per_step": prob.b * prob.m * 2, "d2h_bytes_per_step": prob.b * prob.n * 2,
             "host_issue_us_per_step": round(host_s / K * 1e6, 2),
-            "path": ("twq.DecodeStep -> twq_fused_linear_x_host (H2D, layer, D2H in one C-ABI "
-                     "call), eager, four streams in rotation" if prob.one_launch else
-                     "python binding, eager launches")}
+            "c_abi_calls_per_step": len(xparts), "path": path}
 
 
-def sweep(args, device, peaks):
+def sweep(args, device, peaks, int8_peak=None):
     """Kernel-level numbers of the other workloads: fused, w4a4_only and unfused."""
     import torch
     from rank_residual_w4a4_b200 import twq
@@ -523,7 +632,6 @@ def sweep(args, device, peaks):
     for name in names:
         prob = Problem(name, device)
         wl, b = describe(name)
-        steps = 64 if b <= 64 else 8
         ws = torch.empty(twq.unfused_workspace_bytes(b, wl.n, wl.r), dtype=torch.uint8, device=device)
         res = {"workload": name, "b": b, "m": wl.m, "n": wl.n, "r": wl.r}
 
@@ -568,22 +676,25 @@ def sweep(args, device, peaks):
             quant(i)
             quant8(i)
         torch.cuda.synchronize()
-        t_f = kernel_only_time(prob, fused, steps, reps=3)
-        t_w = kernel_only_time(prob, w4, steps, reps=3)
-        t_u = kernel_only_time(prob, unf, steps, reps=3)
-        t_q = kernel_only_time(prob, quant, steps, reps=3)
-        t_x = kernel_only_time(prob, prob.step_x, steps, reps=3) if prob.one_launch else None
-        t_a8 = kernel_only_time(prob, prob.step_x_a8, steps, reps=3) if prob.one_launch else None
-        t_f8 = kernel_only_time(prob, fused8, steps, reps=3)
-        t_s2q = kernel_only_time(prob, fused_s2q, steps, reps=3) if s2q else None
+        t_f = kernel_only_time(prob, fused)
+        t_w = kernel_only_time(prob, w4)
+        t_u = kernel_only_time(prob, unf)
+        t_q = kernel_only_time(prob, quant)
+        t_x = kernel_only_time(prob, prob.step_x) if prob.one_launch else None
+        t_a8 = kernel_only_time(prob, prob.step_x_a8) if prob.one_launch else None
+        t_f8 = kernel_only_time(prob, fused8)
+        t_s2q = kernel_only_time(prob, fused_s2q) if s2q else None
         ops = int8_ops(b, wl.m, wl.n, wl.r) + bf16_flops(b, wl.n, wl.r)
         res.update({
             "fused_us": round(t_f * 1e6, 2), "w4a4_only_us": round(t_w * 1e6, 2),
             "unfused_us": round(t_u * 1e6, 2), "quantize_us": round(t_q * 1e6, 2),
             "fused_tops": round(ops / t_f / 1e12, 2), "tokens_per_s": round(b / (t_f + t_q), 1),
             "lowrank_overhead": round(t_f / t_w - 1.0, 4), "fusion_speedup": round(t_u / t_f, 3),
-            "roofline": roofline_entry(name, t_f, peaks, profiled_traffic(name)),
-            "timing": "graph of back-to-back launches, weights rotating over %d copies" % prob.copies,
+            "roofline": roofline_entry(name, t_f, peaks, profiled_traffic(name),
+                                       int8_measured=int8_peak),
+            "timing": "median over %d replays of a graph of %d back-to-back launches, weights "
+                      "rotating over %d copies" % (launch_plan(prob)[1], launch_plan(prob)[0],
+                                                  prob.copies),
             "w4a8_fused_us": round(t_f8 * 1e6, 2),
             "w4a8_roofline": roofline_entry(name, t_f8, peaks, None),
         })
@@ -658,10 +769,12 @@ class OracleProblem:
         self.L2 = L2
 
     def rows(self, rows):
+        """Y (BF16 bits) of the given rows, from BF16 X through the oracle's quantizer."""
         import oracle
         xr = self.x[rows]
         qx, sx = oracle.quantize_rows(xr)
-        oracle.linear(qx, sx, self.qr, self.sr, self.ql1, self.sl1, self.L2, mode=oracle.FUSED)
+        return oracle.linear(qx, sx, self.qr, self.sr, self.ql1, self.sl1, self.L2,
+                             mode=oracle.FUSED)["y"]
 
 
 def oracle_rows_parallel(op, row_lists):
@@ -672,24 +785,77 @@ def oracle_rows_parallel(op, row_lists):
         t.join()
 
 
-def cpu_baseline(name, seconds=10.0):
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def compare_rows(y_dev_bits, y_ref_bits):
+    """The tests' Y tolerance: relative Frobenius error <= 2e-3 and per element
+    |dY| <= 1e-2 rms(Y_ref) + 1 BF16 ulp of Y_ref (both against the oracle's BF16 Y)."""
+    f = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    yd, yr = f(y_dev_bits), f(y_ref_bits)
+    rms = float(np.sqrt(np.mean(yr ** 2)))
+    frob = float(np.linalg.norm(yd - yr) / max(np.linalg.norm(yr), 1e-300))
+    a = np.maximum(np.abs(yr), 2.0 ** -126)
+    ulp = 2.0 ** (np.floor(np.log2(a)) - 7)
+    excess = float((np.abs(yd - yr) - (1e-2 * rms + ulp)).max())
+    ok = bool(np.isfinite(yd).all() and frob <= 2e-3 and excess <= 0.0)
+    return {"ok": ok, "rows": int(y_dev_bits.shape[0]), "rel_frobenius": frob,
+            "max_excess_over_elem_bound": excess}
+
+
+def cpu_baseline(name, seconds=10.0, check=None):
+    """The oracle timed on the host cores: a single-core leg and an all-cores leg (rows
+    split over os.cpu_count() threads, each running the unmodified single-threaded
+    oracle on its own rows), each about `seconds` long. With `check` = (rows, GPU Y
+    bits of those rows), the oracle's Y of the same rows is compared with the GPU's."""
     op = OracleProblem(name)
     cores = os.cpu_count() or 1
-    # calibrate on one row per core
+    out = {"unit": "tokens/s", "cores": cores, "kind": "oracle", "cpu_model": cpu_model()}
+    if check is not None:
+        rows, y_dev = check
+        parts = np.array_split(np.arange(rows.size), min(cores, rows.size))
+        res = [None] * len(parts)
+
+        def work(k):
+            res[k] = op.rows(rows[parts[k]])
+
+        threads = [threading.Thread(target=work, args=(k,)) for k in range(len(parts))]
+        for t in threads:
+            t.start()
+        for t in threads:
+            t.join()
+        out["output_check"] = compare_rows(y_dev, np.concatenate(res, axis=0))
+    # single core: calibrate on one row, then about `seconds` of rows
     t0 = time.time()
-    oracle_rows_parallel(op, [np.array([i % op.b]) for i in range(cores)])
-    per_round = max(time.time() - t0, 1e-6)
-    rounds = max(1, int(seconds / per_round))
-    rows_per_thread = rounds
+    op.rows(np.array([0]))
+    per_row = max(time.time() - t0, 1e-6)
+    n1 = max(1, int(seconds / per_row))
+    t0 = time.time()
+    op.rows(np.arange(n1) % op.b)
+    t1 = time.time() - t0
+    out["single_core"] = {"value": round(n1 / t1, 3), "unit": "tokens/s", "cores": 1,
+                          "rows": n1}
+    # all cores
+    rows_per_thread = max(1, int(seconds / per_row))
     lists = [np.arange(i * rows_per_thread, (i + 1) * rows_per_thread) % op.b for i in range(cores)]
     t0 = time.time()
     oracle_rows_parallel(op, lists)
     t = time.time() - t0
     nrows = rows_per_thread * cores
-    return {"value": round(nrows / t, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "%d rows of the %s workload (cycled over its %d tokens), %d threads each "
-                      "running the single-threaded oracle on its own rows; weights quantized "
-                      "outside the timing" % (nrows, name, op.b, cores)}
+    out["value"] = round(nrows / t, 3)
+    out["sample"] = ("all-cores leg: %d rows of the %s workload (cycled over its %d tokens), %d "
+                     "threads each running the single-threaded oracle on its own rows; single-core "
+                     "leg: %d rows on one thread; weights quantized outside the timing" % (
+                         nrows, name, op.b, cores, n1))
+    return out
 
 
 def run_reference(args):
@@ -723,13 +889,57 @@ def run_reference(args):
                    "b": b, "m": wl.m, "n": wl.n, "r": wl.r, "parallelism": "host threads"},
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
-                         "kind": "oracle",
+                         "kind": "oracle", "cpu_model": cpu_model(),
                          "sample": "each step: %d rows of the %s workload over %d threads" % (
                              rows_per_step, name, cores)},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_profile(args):
+    """A plain run for profilers: one copy of the workload's inputs, W + K eager calls
+    of one entry point, no timing. The command lines under profiles/ use it."""
+    import torch
+    from rank_residual_w4a4_b200 import _build, twq
+    _build.build()
+    twq.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    prob = Problem(args.workload, device, copies=1)
+    kind = args.profile
+    b, m = prob.b, prob.m
+    w, x, xq, sx, y = prob.weights[0], prob.x[0], prob.xq[0], prob.sx[0], prob.y[0]
+    twq.quantize_act(x, xq, sx)
+    extra = {}
+    if kind == "a8":
+        extra["xq8"], extra["sx8"] = twq.quantize_act_a8(x)
+    if kind == "s2q":
+        extra["l2q"], extra["sl2q"] = twq.pack_l2_int4(w.l2t.t().contiguous())
+    if kind == "unfused":
+        extra["ws"] = torch.empty(twq.unfused_workspace_bytes(b, prob.n, prob.r), dtype=torch.uint8,
+                                  device=device)
+    torch.cuda.synchronize()
+    calls = {
+        "step": lambda: prob.step(0),
+        "quant": lambda: twq.quantize_act(x, xq, sx),
+        "fused": lambda: twq.fused_linear(xq, sx, w, y),
+        "w4a4": lambda: twq.w4a4_only(xq, sx, w, y),
+        "lowrank": lambda: twq.lowrank_only(xq, sx, w, y),
+        "fused_x": lambda: twq.fused_linear_x(x, w, y),
+        "a8": lambda: twq.fused_linear_a8(extra["xq8"], extra["sx8"], w, y),
+        "s2q": lambda: twq.fused_linear_s2q(xq, sx, w, extra["l2q"], extra["sl2q"], y),
+        "unfused": lambda: twq.unfused_linear(xq, sx, w, y, extra["ws"]),
+    }
+    for _ in range(args.warmup + args.steps):
+        calls[kind]()
+    torch.cuda.synchronize()
+    st = twq.device_status()
+    print(json.dumps({"profile": kind, "workload": args.workload, "calls": args.warmup + args.steps,
+                      "device_status": st}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
 
 
 def main():
@@ -745,7 +955,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--clock-seconds", type=float, default=1.0,
                     help="seconds of warm-up replays before the timed region (clock sampling)")
+    ap.add_argument("--profile", choices=["step", "quant", "fused", "w4a4", "lowrank", "fused_x",
+                                          "a8", "s2q", "unfused"],
+                    help="plain run for a profiler: W + K eager calls of one entry point on one "
+                         "copy of the inputs, no timing")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -196,6 +196,28 @@ TWQ_API twq_status twq_fused_linear_x_host(const uint16_t* x_host, int64_t b, co
                                            twq_stream_t stream);
 
 /*
+ * One layer call from host memory to host memory for any batch (TwinQuant §4.3:
+ * the activation is quantized once and feeds both GEMMs of the fused layer;
+ * this is the call a user makes with the activations in host memory). On
+ * `stream`, in order:
+ *   1. copy x_host (b x m BF16, row-major, contiguous) into x_dev;
+ *   2. batches that twq_fused_linear_x takes (1 <= b <= 16, r <= 128,
+ *      m <= 8192): that one-launch layer on x_dev (xq, sx are not touched and
+ *      may be NULL); any other batch: twq_quantize_act of x_dev into xq (b x m/2
+ *      bytes) and sx (b x m/128 fp32), then twq_fused_linear into y_dev;
+ *   3. copy y_dev (b x n BF16) into y_host.
+ * Nothing is synchronized; y_host holds the result once the stream reaches the
+ * end of the call. Host buffers should be page-locked, or the copies are not
+ * asynchronous. The caller owns every buffer; x_dev, xq, sx and y_dev must not
+ * be in use by other streams while the call runs. Errors: the checks of the
+ * calls it makes, all before anything is enqueued; TWQ_ERR_CUDA if enqueueing
+ * a copy or a launch fails.
+ */
+TWQ_API twq_status twq_linear_host(const uint16_t* x_host, int64_t b, const twq_weights* w,
+                                   uint16_t* x_dev, uint8_t* xq, float* sx, uint16_t* y_dev,
+                                   uint16_t* y_host, twq_stream_t stream);
+
+/*
  * W4A8: 4-bit weights with 8-bit activations, the second quantization setting
  * of TwinQuant §5.1. The activations use Eq. (1) with k = 8 (q_max = 127), in
  * groups of 128 along m with one FP32 scale per token and group; the weights
@@ -289,9 +311,12 @@ TWQ_API twq_status twq_unfused_linear(const uint8_t* xq, const float* sx, int64_
  *   object that every GPU which loads the library holds until the process
  *   exits). Calls whose twq_unfused_workspace_bytes(b, n, r) exceeds 16 MiB
  *   return TWQ_ERR_UNSUPPORTED and launch nothing.
+ *   With w->r == 0 the comparator is the W4A4 kernel alone (twq_w4a4_only),
+ *   which uses no scratch, so the 16 MiB limit does not apply.
  *   Set-up: the first call on each device resolves the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture. The address is kept until twq_release_cache():
+ *   after a cudaDeviceReset, call twq_release_cache() before the next call.
  *   Sharing: every call uses the same array, which keeps the last call's
  *   contents. No part of it needs to start at zero (each call writes every
  *   scratch byte before reading it), but calls that overlap on the GPU (two
@@ -332,6 +357,20 @@ TWQ_API twq_status twq_fold_transforms(const float* Q, const float* G, const uin
  * a site code (which wait gave up). Returns TWQ_ERR_DEVICE if *code != 0.
  */
 TWQ_API twq_status twq_device_status(int* code);
+
+/*
+ * Drops the library's host-side caches: the encoded TMA tensor maps of the
+ * decode path (a direct-mapped table of 256 entries keyed by base pointer,
+ * shape, stride and box; an entry only encodes an address and a shape, so a hit
+ * is always exact and the table never needs clearing for correctness) and the
+ * resolved device addresses of twq_unfused_linear_noalloc's scratch array.
+ * After a cudaDeviceReset in the caller's process, call this before the next
+ * call into the library: the reset ends the context that the cached scratch
+ * address belonged to. Host only; launches nothing; safe to call at any time
+ * from any thread (calls in flight on other threads keep the entries they
+ * already read).
+ */
+TWQ_API void twq_release_cache(void);
 
 /* Number of kernels each entry point launches (for launch accounting). */
 TWQ_API int twq_launches_per_call(const char* entry_point);

@@ -264,6 +264,44 @@ twq_status twq_fused_linear_x_host(const uint16_t* x_host, int64_t b, const twq_
   return TWQ_OK;
 }
 
+twq_status twq_linear_host(const uint16_t* x_host, int64_t b, const twq_weights* w,
+                           uint16_t* x_dev, uint8_t* xq, float* sx, uint16_t* y_dev,
+                           uint16_t* y_host, twq_stream_t stream) {
+  if (!w) return TWQ_ERR_INVALID_ARG;
+  twq_status s = shape_ok(w->m, w->n, w->r);
+  if (s != TWQ_OK) return s;
+  if (b < 0) return TWQ_ERR_INVALID_ARG;
+  if (b > (int64_t(1) << 30)) return TWQ_ERR_UNSUPPORTED;
+  if (b == 0) return TWQ_OK;
+  if (!x_host || !y_host || !x_dev || !y_dev) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(x_dev)) return TWQ_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(b) * w->m * 2, yb = static_cast<size_t>(b) * w->n * 2;
+  // Decode batches that the one-launch layer takes: no codes in HBM at all.
+  twq::GemmCall c{};
+  const bool one = prepare_fused_x(x_dev, w->m, b, w, y_dev, &c) == TWQ_OK;
+  if (!one) {
+    const bool lr = w->r > 0;
+    if ((s = check_layer(xq, sx, b, w, y_dev, true, lr)) != TWQ_OK) return s;
+  }
+  if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return TWQ_ERR_CUDA;
+  cudaError_t e;
+  if (one) {
+    e = twq::launch_decode(c, st);
+  } else {
+    e = twq::launch_quantize_act(x_dev, b, w->m, w->m, xq, sx, st);
+    if (e == cudaSuccess) {
+      s = run(w->r > 0 ? twq::kModeFused : twq::kModeW4A4, xq, sx, b, w, y_dev, nullptr, stream);
+      if (s != TWQ_OK) return s;
+    }
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  if (cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return TWQ_ERR_CUDA;
+  return TWQ_OK;
+}
+
 size_t twq_unfused_workspace_bytes(int64_t b, int64_t n, int64_t r) {
   if (b <= 0 || n <= 0 || r < 0) return 0;
   // Y_res fp32 (b x n) | Y_lr fp32 (b x n) | H bf16 (b x r), each 256-byte aligned
@@ -306,6 +344,11 @@ twq_status twq_device_status(int* code) {
   return *code ? TWQ_ERR_DEVICE : TWQ_OK;
 }
 
+void twq_release_cache(void) {
+  twq::release_decode_cache();
+  twq::release_noalloc_cache();
+}
+
 int twq_launches_per_call(const char* ep) {
   if (!ep) return -1;
   if (!strcmp(ep, "twq_quantize_act") || !strcmp(ep, "twq_quantize_act_a8")) return 1;
@@ -316,6 +359,7 @@ int twq_launches_per_call(const char* ep) {
       !strcmp(ep, "twq_fused_linear_x_host") || !strcmp(ep, "twq_fused_linear_a8") ||
       !strcmp(ep, "twq_fused_linear_x_a8"))
     return 1;
+  if (!strcmp(ep, "twq_linear_host")) return 2;  // 1 for the batches twq_fused_linear_x takes
   if (!strcmp(ep, "twq_unfused_linear") || !strcmp(ep, "twq_unfused_linear_noalloc")) return 4;
   if (!strcmp(ep, "twq_fold_transforms")) return 5;
   return -1;

@@ -375,6 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the stage-2 B tile (H's codes) is zero beyond the CTA's slice of r (K padding)
       for (int e = lane; e < 2048 / 16; e += 32)
         reinterpret_cast<uint4*>(hbs)[e] = make_uint4(0, 0, 0, 0);
+      // the MMAs read this tile through the async proxy: order the generic-proxy
+      // zero-fill before them (the CTA barrier below then publishes it)
+      fence_proxy_async_smem();
     }
     fence_barrier_init();
     __syncwarp();
@@ -894,6 +897,12 @@ bool d_encode_raw(CUtensorMap* map, CUtensorMapDataType dt, const void* base, ui
                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                   CUtensorMapSwizzle sw);
 
+// Drops every cached map (twq_release_cache).
+void clear_map_cache() {
+  std::lock_guard<std::mutex> lock(g_map_mutex);
+  for (MapEntry& e : g_map_cache) e.valid = false;
+}
+
 bool d_encode(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
               CUtensorMapSwizzle sw) {
@@ -1055,5 +1064,7 @@ cudaError_t read_and_clear_decode_status(int* code) {
   *code = v;
   return e;
 }
+
+void release_decode_cache() { clear_map_cache(); }
 
 }  // namespace twq

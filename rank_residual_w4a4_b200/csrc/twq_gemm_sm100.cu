@@ -28,6 +28,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "sm100_ptx.cuh"
 #include "twq_eq1.cuh"
@@ -1045,7 +1046,9 @@ int num_sms() {
 // per instantiation (0 if the query fails: no pairs then).
 template <int kMode, int BN, bool kA8>
 int resident_pairs() {
-  static int cached = -1;
+  // Concurrent first calls may both run the query; they store the same value.
+  static std::atomic<int> cached_atomic{-1};
+  int cached = cached_atomic.load(std::memory_order_acquire);
   if (cached < 0) {
     using L = SmemLayout<BN, kA8>;
     auto kern = twq_gemm_kernel<kMode, BN, true, kA8>;
@@ -1071,6 +1074,7 @@ int resident_pairs() {
       (void)cudaGetLastError();
     }
     cached = nc > 0 ? nc : 0;
+    cached_atomic.store(cached, std::memory_order_release);
   }
   return cached;
 }

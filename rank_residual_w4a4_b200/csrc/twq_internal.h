@@ -50,6 +50,11 @@ cudaError_t launch_add_cast(const float* a, const float* b, int64_t count, uint1
 bool decode_eligible(const GemmCall& call);
 cudaError_t launch_decode(const GemmCall& call, cudaStream_t stream);
 
+// twq_release_cache: drop the decode path's cached tensor maps, and the
+// allocation-free entry point's resolved scratch addresses.
+void release_decode_cache();
+void release_noalloc_cache();
+
 // Device status words (first wait site that gave up), one per kernel family.
 cudaError_t read_and_clear_device_status(int* code);
 cudaError_t read_and_clear_decode_status(int* code);

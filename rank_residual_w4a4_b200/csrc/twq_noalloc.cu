@@ -43,12 +43,25 @@ twq_status scratch_address(void** out) {
 
 }  // namespace
 
+namespace twq {
+// Forgets the resolved addresses, so that the next call on each device resolves
+// the array again (needed after the caller's cudaDeviceReset, which ends the
+// context that the old address belonged to).
+void release_noalloc_cache() {
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  for (void*& p : g_scratch_addr) p = nullptr;
+}
+}  // namespace twq
+
 extern "C" twq_status twq_unfused_linear_noalloc(const uint8_t* xq, const float* sx, int64_t b,
                                                  const twq_weights* w, uint16_t* y,
                                                  twq_stream_t stream) {
   if (!w || b < 0) return TWQ_ERR_INVALID_ARG;
   if (b == 0) return twq_unfused_linear(xq, sx, b, w, y, nullptr, 0, stream);
   if (w->m <= 0 || w->n <= 0 || w->r < 0) return TWQ_ERR_INVALID_ARG;
+  // Without a low-rank part the comparator is the W4A4 kernel alone (what
+  // twq_unfused_linear runs for r == 0), which uses no scratch: no size limit then.
+  if (w->r == 0) return twq_w4a4_only(xq, sx, b, w, y, stream);
   const size_t need = twq_unfused_workspace_bytes(b, w->n, w->r);
   if (need == 0) return TWQ_ERR_INVALID_ARG;
   if (need > kNoAllocScratchBytes) return TWQ_ERR_UNSUPPORTED;  // beyond the fixed 16 MiB

@@ -29,7 +29,8 @@ EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_siz
            "twq_device_status", "twq_launches_per_call", "twq_unfused_linear_noalloc",
            "twq_fused_linear_x", "twq_fold_workspace_bytes", "twq_fold_transforms",
            "twq_fused_linear_x_host", "twq_quantize_act_a8", "twq_fused_linear_a8",
-           "twq_fused_linear_x_a8", "twq_pack_l2_int4", "twq_fused_linear_s2q")
+           "twq_fused_linear_x_a8", "twq_pack_l2_int4", "twq_fused_linear_s2q",
+           "twq_linear_host", "twq_release_cache")
 
 
 class TwqError(RuntimeError):
@@ -81,6 +82,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twq_fused_linear_s2q": ([P, P, I, P, P, P, P, P], ctypes.c_int),
         "twq_fold_workspace_bytes": ([I, I, I], S),
         "twq_fold_transforms": ([P, P, P, P, P, I, I, I, P, P, P, P, S, P], ctypes.c_int),
+        "twq_linear_host": ([P, I, P, P, P, P, P, P, P], ctypes.c_int),
+        "twq_release_cache": ([], None),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -339,6 +342,46 @@ class DecodeStep:
         _check(self._fn(x_host.data_ptr(), self._b, ctypes.byref(w.c_struct()), self._xd, self._yd,
                         self._yh, self._st), "twq_fused_linear_x_host")
         return self.y_host
+
+
+class LinearHostStep:
+    """A prepared twq_linear_host call: one layer call for any batch from host memory
+    to host memory (H2D copy of X, the quantizer and the fused layer, or the one-launch
+    layer for decode batches, D2H copy of Y), all enqueued on one stream by one C call.
+    The device buffers (X, codes, scales, Y), the pinned host output and the stream are
+    checked once."""
+
+    def __init__(self, b: int, m: int, n: int, device, stream=None, y_host: torch.Tensor | None = None):
+        self._b, self._m, self._n = b, m, n
+        self.x_dev = torch.empty((b, m), dtype=torch.bfloat16, device=device)
+        self.xq = torch.empty((b, m // 2), dtype=torch.uint8, device=device)
+        self.sx = torch.empty((b, max(m // 128, 1)), dtype=torch.float32, device=device)
+        self.y_dev = torch.empty((b, n), dtype=torch.bfloat16, device=device)
+        if y_host is None:
+            y_host = torch.empty((b, n), dtype=torch.bfloat16).pin_memory()
+        if y_host.is_cuda or y_host.dtype != torch.bfloat16 or not y_host.is_contiguous() \
+                or tuple(y_host.shape) != (b, n):
+            raise TypeError("y_host must be a contiguous host torch.bfloat16 tensor of shape (b, n)")
+        self.y_host = y_host
+        self._ptrs = (self.x_dev.data_ptr(), self.xq.data_ptr(), self.sx.data_ptr(),
+                      self.y_dev.data_ptr(), y_host.data_ptr())
+        self._st = _stream(stream)
+        self._fn = load().twq_linear_host
+
+    def __call__(self, x_host: torch.Tensor, w: Weights) -> torch.Tensor:
+        if x_host.is_cuda or x_host.dtype != torch.bfloat16 or not x_host.is_contiguous():
+            raise TypeError("x_host must be a contiguous host torch.bfloat16 tensor")
+        if tuple(x_host.shape) != (self._b, self._m) or w.m != self._m or w.n != self._n:
+            raise ValueError("x_host and w must match the prepared shapes")
+        xd, xq, sx, yd, yh = self._ptrs
+        _check(self._fn(x_host.data_ptr(), self._b, ctypes.byref(w.c_struct()), xd, xq, sx, yd,
+                        yh, self._st), "twq_linear_host")
+        return self.y_host
+
+
+def release_cache() -> None:
+    """Drop the library's host-side caches (call after a cudaDeviceReset)."""
+    load().twq_release_cache()
 
 
 def fold_workspace_bytes(m: int, n: int, r: int) -> int:

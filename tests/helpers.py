@@ -12,6 +12,18 @@ FROB_TOL = 2e-3
 ELEM_TOL = 1e-2
 
 
+def block_rows(b, per_block=2, seed=0, block=128):
+    """Seeded rows of a b-row output, `per_block` from every `block`-row block (so every
+    row block of the kernels' schedules is compared), plus the last row."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for r0 in range(0, b, block):
+        hi = min(b, r0 + block)
+        rows.extend(rng.choice(np.arange(r0, hi), size=min(per_block, hi - r0), replace=False))
+    rows.append(b - 1)
+    return np.unique(np.array(rows, dtype=np.int64))
+
+
 def to_dev(a, dev):
     import torch
     a = np.ascontiguousarray(a)

@@ -88,3 +88,40 @@ def test_reference_arm_prints_the_contract_line():
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert "workload" in line["config"]
+
+
+def test_sample_rows_cover_every_row_block():
+    for b in (1, 16, 129, 2048, 8192):
+        rows = bench.sample_rows(b)
+        assert rows.min() >= 0 and rows.max() == b - 1
+        assert set(rows // 128) == set(range((b + 127) // 128))
+
+
+def test_output_check_flags_a_wrong_row():
+    import numpy as np
+    rng = np.random.default_rng(1)
+    y = rng.standard_normal((4, 256)).astype(np.float32)
+    bits = (y.view(np.uint32) >> 16).astype(np.uint16)  # truncation: within one ulp
+    assert bench.compare_rows(bits, bits)["ok"]
+    bad = bits.copy()
+    bad[2, 7] ^= 0x4000  # a large error in one element
+    assert not bench.compare_rows(bad, bits)["ok"]
+
+
+def test_kernel_timing_covers_at_least_200_launches():
+    class P:
+        pass
+    for b, copies in ((16, 26), (8192, 4), (2048, 2)):
+        p = P()
+        p.b, p.copies = b, copies
+        per, replays = bench.launch_plan(p)
+        assert per % copies == 0 and per * replays >= bench.MIN_TIMED_LAUNCHES and replays >= 5
+
+
+def test_gpus_flag_must_match_the_launched_ranks(monkeypatch):
+    import sys
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "2", "--steps", "3", "--warmup", "3"])
+    with pytest.raises(SystemExit) as e:
+        bench.main()
+    assert "ranks" in str(e.value)

@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import synth
-from helpers import assert_y_close, bits_of, to_dev
+from helpers import assert_y_close, bits_of, block_rows, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -326,6 +326,8 @@ def test_workload_all_rows(twq, device, name, b):
 
 
 @pytest.mark.parametrize("name", ["gateup", "down", "large"])
-def test_workload_sampled_rows(twq, device, name):
+def test_workload_rows_of_every_row_block(twq, device, name):
+    """Full-size prefill workloads: two seeded rows of every 128-row block (every row
+    block of the persistent schedule, so every CTA's work), all columns."""
     wl = synth.WORKLOADS[name]
-    _full(twq, device, name, wl.b, synth.sample_rows(wl.b, 24, seed=11))
+    _full(twq, device, name, wl.b, block_rows(wl.b, per_block=2, seed=11))

@@ -48,13 +48,41 @@ def _call_noalloc(lib, w, xq, sx):
 
 
 def test_noalloc_matches_workspace_version_twice(lib, device):
+    """Same kernels and arithmetic as twq_unfused_linear, so the results are bitwise
+    equal (which is within the tests' Y tolerance too)."""
     from rank_residual_w4a4_b200 import twq
     for shape, seed in (((200, 512, 384, 144), 21), ((33, 256, 256, 32), 22)):
         w, xq, sx = _case(device, *shape, seed=seed)
         y_ref = twq.unfused_linear(xq, sx, w)
         y = _call_noalloc(lib, w, xq, sx)
         torch.cuda.synchronize()
+        assert np.array_equal(bits_of(y), bits_of(y_ref)), "noalloc %s" % (shape,)
         assert_y_close(bits_of(y), bits_of(y_ref), "noalloc %s" % (shape,))
+    assert twq.device_status() == 0
+
+
+def test_noalloc_without_low_rank_has_no_size_limit(lib, device):
+    """r == 0: the comparator is the W4A4 kernel alone, which uses no scratch, so a batch
+    whose fp32 intermediates would not fit in the fixed array still runs."""
+    from rank_residual_w4a4_b200 import twq
+    w, xq, sx = _case(device, 4096, 256, 1024, 0, seed=23)  # 4096 x 1024 x 8 B = 32 MiB
+    y = _call_noalloc(lib, w, xq, sx)
+    y_ref = twq.unfused_linear(xq, sx, w)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits_of(y), bits_of(y_ref))
+    assert twq.device_status() == 0
+
+
+def test_noalloc_after_release_cache(lib, device):
+    """twq_release_cache() forgets the resolved scratch address; the next call resolves it
+    again and gives the same result."""
+    from rank_residual_w4a4_b200 import twq
+    w, xq, sx = _case(device, 64, 256, 256, 32, seed=24)
+    y0 = _call_noalloc(lib, w, xq, sx)
+    lib.twq_release_cache()
+    y1 = _call_noalloc(lib, w, xq, sx)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits_of(y0), bits_of(y1))
     assert twq.device_status() == 0
 
 

@@ -258,6 +258,10 @@ class Problem:
         self.x = [xd] + [xd.clone() for _ in range(copies - 1)]
         self.xq = [torch.empty((b, self.m // 2), dtype=torch.uint8, device=device)
                    for _ in range(copies)]
+        # prefill: the same codes one per byte (twq_quantize_act_i8), which the layer
+        # kernel reads as they lie
+        self.xq8 = ([torch.empty((b, self.m), dtype=torch.int8, device=device)
+                     for _ in range(copies)] if b > 16 else None)
         self.sx = [torch.empty((b, self.m // 128), dtype=torch.float32, device=device)
                    for _ in range(copies)]
         self.y = [torch.empty((b, self.n), dtype=torch.bfloat16, device=device) for _ in range(copies)]
@@ -272,7 +276,14 @@ class Problem:
         if self.one_launch:
             self.step_x(i)
         else:
-            self.step_two_call(i)
+            self.step_bytes(i)
+
+    def step_bytes(self, i):
+        """Prefill: twq_quantize_act_i8 + twq_fused_linear_i8 (the codes one per byte)."""
+        from rank_residual_w4a4_b200 import twq
+        c = i % self.copies
+        twq.quantize_act_i8(self.x[c], self.xq8[c], self.sx[c])
+        twq.fused_linear_i8(self.xq8[c], self.sx[c], self.weights[c], self.y[c])
 
     def step_x(self, i):
         from rank_residual_w4a4_b200 import twq
@@ -458,16 +469,18 @@ def run_gpu(args):
     # back-to-back launches on the same stream and weight rotation
     def fused_only(i):
         c = i % prob.copies
-        twq.fused_linear(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c])
+        twq.fused_linear_i8(prob.xq8[c], prob.sx[c], prob.weights[c], prob.y[c])
 
     def quant_only(i):
         c = i % prob.copies
-        twq.quantize_act(prob.x[c], prob.xq[c], prob.sx[c])
+        twq.quantize_act_i8(prob.x[c], prob.xq8[c], prob.sx[c])
 
     one = prob.one_launch
     t_fused = kernel_only_time(prob, prob.step_x if one else fused_only)
     t_quant = None if one else kernel_only_time(prob, quant_only)
-    t_two = time_graph(capture(prob.step_two_call, K), world, device) / K if one else None
+    # the two-call step on packed codes (twq_quantize_act + twq_fused_linear), for
+    # decode and prefill batches alike
+    t_two = time_graph(capture(prob.step_two_call, K), world, device) / K
     t_a8 = time_graph(capture(prob.step_x_a8, K), world, device) / K if one else None
     st = twq.device_status()
     if st != 0:
@@ -508,7 +521,9 @@ def run_gpu(args):
         "config": {"workload": "%s: b=%d m=%d n=%d r=%d, group 128" % (name, b, wl.m, wl.n, wl.r),
                    "b": b, "m": wl.m, "n": wl.n, "r": wl.r, "parallelism": "replicas x%d" % world,
                    "step": ("twq_fused_linear_x (activation quantizer inside the layer kernel)"
-                            if one else "twq_quantize_act + twq_fused_linear"),
+                            if one else "twq_quantize_act_i8 + twq_fused_linear_i8 (the 4-bit "
+                            "activation codes stored one per byte; bitwise the Y of "
+                            "twq_quantize_act + twq_fused_linear)"),
                    "l2": "inputs larger than L2: weights rotate over %d copies (%.0f MB > 2x L2); "
                          "X %.0f MB and Y %.0f MB per step" % (
                              prob.copies, prob.copies * weight_bytes(wl.m, wl.n, wl.r) / 1e6,
@@ -536,9 +551,10 @@ def run_gpu(args):
                                      "peak": peaks[0], "unit": "GB/s",
                                      "frac": round(qb / t_quant / 1e9 / peaks[0], 4),
                                      "algorithmic_bytes": qb}
+    line["two_call_step_us"] = round(t_two * 1e6, 3)
+    line["two_call_step"] = ("twq_quantize_act + twq_fused_linear (packed 4-bit activation "
+                             "codes), same graph timing")
     if one:
-        line["two_call_step_us"] = round(t_two * 1e6, 3)
-        line["two_call_step"] = "twq_quantize_act + twq_fused_linear, same graph timing"
         line["w4a8_step_us"] = round(t_a8 * 1e6, 3)
         line["w4a8_step"] = ("twq_fused_linear_x_a8: the same layer with 8-bit activation codes "
                              "(W4A8), same graph timing")
@@ -635,13 +651,35 @@ def sweep(args, device, peaks, int8_peak=None):
         ws = torch.empty(twq.unfused_workspace_bytes(b, wl.n, wl.r), dtype=torch.uint8, device=device)
         res = {"workload": name, "b": b, "m": wl.m, "n": wl.n, "r": wl.r}
 
-        def fused(i):
+        prefill = b > 16
+
+        def fused_packed(i):
             c = i % prob.copies
             twq.fused_linear(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c])
 
-        def w4(i):
+        def w4_packed(i):
             c = i % prob.copies
             twq.w4a4_only(prob.xq[c], prob.sx[c], prob.weights[c], prob.y[c])
+
+        # prefill: the layer on the codes stored one per byte, and the same kernel without
+        # the low-rank part (a view of the weights with r = 0), for the low-rank overhead
+        w_r0 = [twq.Weights(wc.m, wc.n, 0, wc.rq, wc.sr, wc.l1q[:0], wc.sl1[:, :0], wc.l2t[:, :0])
+                for wc in prob.weights]
+
+        def fused_b(i):
+            c = i % prob.copies
+            twq.fused_linear_i8(prob.xq8[c], prob.sx[c], prob.weights[c], prob.y[c])
+
+        def w4_b(i):
+            c = i % prob.copies
+            twq.fused_linear_i8(prob.xq8[c], prob.sx[c], w_r0[c], prob.y[c])
+
+        def quant_b(i):
+            c = i % prob.copies
+            twq.quantize_act_i8(prob.x[c], prob.xq8[c], prob.sx[c])
+
+        fused = fused_b if prefill else fused_packed
+        w4 = w4_b if prefill else w4_packed
 
         def unf(i):
             c = i % prob.copies
@@ -675,11 +713,14 @@ def sweep(args, device, peaks, int8_peak=None):
         for i in range(prob.copies):
             quant(i)
             quant8(i)
+            if prefill:
+                quant_b(i)
         torch.cuda.synchronize()
         t_f = kernel_only_time(prob, fused)
         t_w = kernel_only_time(prob, w4)
         t_u = kernel_only_time(prob, unf)
-        t_q = kernel_only_time(prob, quant)
+        t_q = kernel_only_time(prob, quant_b if prefill else quant)
+        t_fp = kernel_only_time(prob, fused_packed) if prefill else t_f
         t_x = kernel_only_time(prob, prob.step_x) if prob.one_launch else None
         t_a8 = kernel_only_time(prob, prob.step_x_a8) if prob.one_launch else None
         t_f8 = kernel_only_time(prob, fused8)
@@ -689,7 +730,12 @@ def sweep(args, device, peaks, int8_peak=None):
             "fused_us": round(t_f * 1e6, 2), "w4a4_only_us": round(t_w * 1e6, 2),
             "unfused_us": round(t_u * 1e6, 2), "quantize_us": round(t_q * 1e6, 2),
             "fused_tops": round(ops / t_f / 1e12, 2), "tokens_per_s": round(b / (t_f + t_q), 1),
-            "lowrank_overhead": round(t_f / t_w - 1.0, 4), "fusion_speedup": round(t_u / t_f, 3),
+            "lowrank_overhead": round(t_f / t_w - 1.0, 4), "fusion_speedup": round(t_u / t_fp, 3),
+            "fused_packed_us": round(t_fp * 1e6, 2),
+            "fused_input": ("the 4-bit codes one per byte (twq_fused_linear_i8); w4a4_only_us: "
+                            "the same kernel with r = 0; fused_packed_us: twq_fused_linear on "
+                            "packed codes; fusion_speedup: unfused over fused_packed (same input)"
+                            if prefill else "packed codes (twq_fused_linear)"),
             "roofline": roofline_entry(name, t_f, peaks, profiled_traffic(name),
                                        int8_measured=int8_peak),
             "timing": "median over %d replays of a graph of %d back-to-back launches, weights "
@@ -707,7 +753,7 @@ def sweep(args, device, peaks, int8_peak=None):
             res["roofline_x"] = roofline_entry(name, t_x, peaks, profiled_traffic(name + "_x"),
                                                bf16_x=True)
         out.append(res)
-        del prob, ws, xq8, sx8, l2qs
+        del prob, ws, xq8, sx8, l2qs, w_r0
         torch.cuda.empty_cache()
     out.append(fold_entry(device))
     st = twq.device_status()
@@ -912,6 +958,9 @@ def run_profile(args):
     b, m = prob.b, prob.m
     w, x, xq, sx, y = prob.weights[0], prob.x[0], prob.xq[0], prob.sx[0], prob.y[0]
     twq.quantize_act(x, xq, sx)
+    xq8 = prob.xq8[0] if prob.xq8 is not None else None
+    if xq8 is not None:
+        twq.quantize_act_i8(x, xq8, sx)
     extra = {}
     if kind == "a8":
         extra["xq8"], extra["sx8"] = twq.quantize_act_a8(x)
@@ -924,7 +973,9 @@ def run_profile(args):
     calls = {
         "step": lambda: prob.step(0),
         "quant": lambda: twq.quantize_act(x, xq, sx),
+        "quant_i8": lambda: twq.quantize_act_i8(x, xq8, sx),
         "fused": lambda: twq.fused_linear(xq, sx, w, y),
+        "fused_i8": lambda: twq.fused_linear_i8(xq8, sx, w, y),
         "w4a4": lambda: twq.w4a4_only(xq, sx, w, y),
         "lowrank": lambda: twq.lowrank_only(xq, sx, w, y),
         "fused_x": lambda: twq.fused_linear_x(x, w, y),
@@ -955,8 +1006,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--clock-seconds", type=float, default=1.0,
                     help="seconds of warm-up replays before the timed region (clock sampling)")
-    ap.add_argument("--profile", choices=["step", "quant", "fused", "w4a4", "lowrank", "fused_x",
-                                          "a8", "s2q", "unfused"],
+    ap.add_argument("--profile", choices=["step", "quant", "quant_i8", "fused", "fused_i8", "w4a4",
+                                          "lowrank", "fused_x", "a8", "s2q", "unfused"],
                     help="plain run for a profiler: W + K eager calls of one entry point on one "
                          "copy of the inputs, no timing")
     args = ap.parse_args()

@@ -158,6 +158,35 @@ TWQ_API twq_status twq_fused_linear(const uint8_t* xq, const float* sx, int64_t 
                             uint16_t* y, twq_stream_t stream);
 
 /*
+ * The 4-bit activation codes stored one per byte, for prefill batches. The codes and
+ * scales are exactly those of twq_quantize_act (TwinQuant Eq. (1), q_max = 7, per
+ * token and group of 128): only their storage differs, element k of a row in byte k
+ * as a two's-complement int8 in [-7, 7], twice the bytes of the packed form
+ * (b x m instead of b x m/2). The layer's tensor-core kernel reads them where its
+ * copy engine puts them, so it unpacks only the weights, which halves its unpack
+ * work; at prefill sizes the extra activation bytes cost far less than that work.
+ *   x    b x m BF16, row stride ldx elements (ldx >= m, ldx % 8 == 0), finite
+ *   xq8  b x m int8 (output);  sx  b x (m/128) fp32 (output)
+ * Errors as twq_quantize_act.
+ */
+TWQ_API twq_status twq_quantize_act_i8(const uint16_t* x, int64_t b, int64_t m, int64_t ldx,
+                                       int8_t* xq8, float* sx, twq_stream_t stream);
+
+/*
+ * The fused layer (as twq_fused_linear) on activation codes stored one per byte:
+ * the 4-bit codes of twq_quantize_act_i8, or the 8-bit codes of W4A8
+ * (twq_quantize_act_a8). Each group's int8 x int4 dot product is exact in the int32
+ * accumulator (|sum| <= 128 * 127 * 7) and scaled per group in FP32, so with 4-bit
+ * codes the result is bitwise that of twq_quantize_act + twq_fused_linear.
+ *   xq8  b x m int8;  sx  b x (m/128) fp32;  w, y, shapes and errors as
+ *   twq_fused_linear. Prefill batches (b > 16, m >= 256, n % 256 == 0) run the
+ *   CTA-pair tensor-core kernel; decode batches the split-K decode kernel.
+ * Same function as twq_fused_linear_a8 (either name).
+ */
+TWQ_API twq_status twq_fused_linear_i8(const int8_t* xq8, const float* sx, int64_t b,
+                                       const twq_weights* w, uint16_t* y, twq_stream_t stream);
+
+/*
  * The fused layer with the activation quantizer inside it, for decode batches
  * (TwinQuant §4.3: the activation is quantized once, on chip, and the codes feed
  * both the residual GEMM and the first low-rank GEMM). Each CTA quantizes its
@@ -203,8 +232,10 @@ TWQ_API twq_status twq_fused_linear_x_host(const uint16_t* x_host, int64_t b, co
  *   1. copy x_host (b x m BF16, row-major, contiguous) into x_dev;
  *   2. batches that twq_fused_linear_x takes (1 <= b <= 16, r <= 128,
  *      m <= 8192): that one-launch layer on x_dev (xq, sx are not touched and
- *      may be NULL); any other batch: twq_quantize_act of x_dev into xq (b x m/2
- *      bytes) and sx (b x m/128 fp32), then twq_fused_linear into y_dev;
+ *      may be NULL); any other batch: twq_quantize_act_i8 of x_dev into xq
+ *      (b x m bytes: the 4-bit codes one per byte) and sx (b x m/128 fp32), then
+ *      twq_fused_linear_i8 into y_dev (the same Y as twq_quantize_act +
+ *      twq_fused_linear, bitwise);
  *   3. copy y_dev (b x n BF16) into y_host.
  * Nothing is synchronized; y_host holds the result once the stream reaches the
  * end of the call. Host buffers should be page-locked, or the copies are not
@@ -214,7 +245,7 @@ TWQ_API twq_status twq_fused_linear_x_host(const uint16_t* x_host, int64_t b, co
  * a copy or a launch fails.
  */
 TWQ_API twq_status twq_linear_host(const uint16_t* x_host, int64_t b, const twq_weights* w,
-                                   uint16_t* x_dev, uint8_t* xq, float* sx, uint16_t* y_dev,
+                                   uint16_t* x_dev, int8_t* xq, float* sx, uint16_t* y_dev,
                                    uint16_t* y_host, twq_stream_t stream);
 
 /*
@@ -357,6 +388,23 @@ TWQ_API twq_status twq_fold_transforms(const float* Q, const float* G, const uin
  * a site code (which wait gave up). Returns TWQ_ERR_DEVICE if *code != 0.
  */
 TWQ_API twq_status twq_device_status(int* code);
+
+/*
+ * Self-test of the kernels' bounded waits (the pages have no counterpart: this
+ * checks the library's failure path without a GPU fault). Launches the prefill
+ * layer kernel on the given W4A4 problem with its X copies withheld and every
+ * wait limited to wait_limit_ns (1 us .. 1 s), so that the waits on X run out:
+ * the kernel records the site of the first wait that gave up, its CTAs let their
+ * copies in flight land, complete their MMAs, free their tensor memory and leave.
+ * The launch itself succeeds; twq_device_status() then reports a nonzero site
+ * code (41..52) and clears it, and later calls on the stream run normally. y is
+ * left unspecified.
+ *   xq, sx, b, w, y  as twq_w4a4_only, with b > 16, w->m >= 256, w->n % 256 == 0
+ *   (TWQ_ERR_UNSUPPORTED otherwise: the prefill kernel does not take the shape).
+ */
+TWQ_API twq_status twq_selftest_wait_timeout(const uint8_t* xq, const float* sx, int64_t b,
+                                             const twq_weights* w, uint16_t* y,
+                                             int64_t wait_limit_ns, twq_stream_t stream);
 
 /*
  * Drops the library's host-side caches: the encoded TMA tensor maps of the

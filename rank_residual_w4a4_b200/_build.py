@@ -15,8 +15,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libtwq.so")
-SOURCES = ["twq_api.cu", "twq_gemm_sm100.cu", "twq_decode_sm100.cu", "twq_quant.cu",
-           "twq_noalloc.cu", "twq_fold.cu"]
+SOURCES = ["twq_api.cu", "twq_gemm_sm100.cu", "twq_pair_sm100.cu", "twq_decode_sm100.cu",
+           "twq_quant.cu", "twq_noalloc.cu", "twq_fold.cu"]
 HEADERS = ["sm100_ptx.cuh", "twq_internal.h", "twq_eq1.cuh"]
 
 NVCC_FLAGS = [

@@ -116,6 +116,17 @@ twq_status twq_quantize_act_a8(const uint16_t* x, int64_t b, int64_t m, int64_t 
                                             reinterpret_cast<cudaStream_t>(stream), true));
 }
 
+twq_status twq_quantize_act_i8(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, int8_t* xq8,
+                               float* sx, twq_stream_t stream) {
+  if (b < 0 || m <= 0 || m % 128 || ldx < m) return TWQ_ERR_INVALID_ARG;
+  if (m > (int64_t(1) << 24) || b > (int64_t(1) << 30)) return TWQ_ERR_UNSUPPORTED;
+  if (b == 0) return TWQ_OK;
+  if (!x || !xq8 || !sx) return TWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq8) || !aligned16(sx) || ldx % 8) return TWQ_ERR_MISALIGNED;
+  return from_cuda(twq::launch_quantize_act(x, b, m, ldx, reinterpret_cast<uint8_t*>(xq8), sx,
+                                            reinterpret_cast<cudaStream_t>(stream), false, true));
+}
+
 twq_status twq_pack_weights(const uint16_t* R, const uint16_t* L1, const uint16_t* L2,
                             const twq_weights* w, twq_stream_t stream) {
   if (!w) return TWQ_ERR_INVALID_ARG;
@@ -169,6 +180,11 @@ twq_status twq_fused_linear_a8(const int8_t* xq8, const float* sx, int64_t b, co
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (twq::decode_eligible(c)) return from_cuda(twq::launch_decode(c, st));
   return from_cuda(twq::launch_gemm(c, st, nullptr));
+}
+
+twq_status twq_fused_linear_i8(const int8_t* xq8, const float* sx, int64_t b, const twq_weights* w,
+                               uint16_t* y, twq_stream_t stream) {
+  return twq_fused_linear_a8(xq8, sx, b, w, y, stream);
 }
 
 twq_status twq_pack_l2_int4(const uint16_t* L2, int64_t r, int64_t n, uint8_t* l2q, float* sl2q,
@@ -265,7 +281,7 @@ twq_status twq_fused_linear_x_host(const uint16_t* x_host, int64_t b, const twq_
 }
 
 twq_status twq_linear_host(const uint16_t* x_host, int64_t b, const twq_weights* w,
-                           uint16_t* x_dev, uint8_t* xq, float* sx, uint16_t* y_dev,
+                           uint16_t* x_dev, int8_t* xq8, float* sx, uint16_t* y_dev,
                            uint16_t* y_host, twq_stream_t stream) {
   if (!w) return TWQ_ERR_INVALID_ARG;
   twq_status s = shape_ok(w->m, w->n, w->r);
@@ -280,6 +296,7 @@ twq_status twq_linear_host(const uint16_t* x_host, int64_t b, const twq_weights*
   // Decode batches that the one-launch layer takes: no codes in HBM at all.
   twq::GemmCall c{};
   const bool one = prepare_fused_x(x_dev, w->m, b, w, y_dev, &c) == TWQ_OK;
+  const uint8_t* xq = reinterpret_cast<const uint8_t*>(xq8);
   if (!one) {
     const bool lr = w->r > 0;
     if ((s = check_layer(xq, sx, b, w, y_dev, true, lr)) != TWQ_OK) return s;
@@ -290,10 +307,13 @@ twq_status twq_linear_host(const uint16_t* x_host, int64_t b, const twq_weights*
   if (one) {
     e = twq::launch_decode(c, st);
   } else {
-    e = twq::launch_quantize_act(x_dev, b, w->m, w->m, xq, sx, st);
+    // the codes one per byte (twq_quantize_act_i8), which the layer reads as they lie
+    e = twq::launch_quantize_act(x_dev, b, w->m, w->m, reinterpret_cast<uint8_t*>(xq8), sx, st,
+                                 false, true);
     if (e == cudaSuccess) {
-      s = run(w->r > 0 ? twq::kModeFused : twq::kModeW4A4, xq, sx, b, w, y_dev, nullptr, stream);
-      if (s != TWQ_OK) return s;
+      twq::GemmCall g{w->r > 0 ? twq::kModeFused : twq::kModeW4A4, xq, sx, b, w, y_dev, nullptr};
+      g.a8 = true;
+      e = twq::decode_eligible(g) ? twq::launch_decode(g, st) : twq::launch_gemm(g, st, nullptr);
     }
   }
   if (e != cudaSuccess) return from_cuda(e);
@@ -336,12 +356,25 @@ twq_status twq_device_status(int* code) {
   if (!code) return TWQ_ERR_INVALID_ARG;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return TWQ_ERR_CUDA;
-  int c1 = 0, c2 = 0;
+  int c1 = 0, c2 = 0, c3 = 0;
   e = twq::read_and_clear_device_status(&c1);
   if (e == cudaSuccess) e = twq::read_and_clear_decode_status(&c2);
+  if (e == cudaSuccess) e = twq::read_and_clear_pair_status(&c3);
   if (e != cudaSuccess) return TWQ_ERR_CUDA;
-  *code = c1 ? c1 : c2;
+  *code = c1 ? c1 : (c2 ? c2 : c3);
   return *code ? TWQ_ERR_DEVICE : TWQ_OK;
+}
+
+twq_status twq_selftest_wait_timeout(const uint8_t* xq, const float* sx, int64_t b,
+                                     const twq_weights* w, uint16_t* y, int64_t wait_limit_ns,
+                                     twq_stream_t stream) {
+  twq_status s = check_layer(xq, sx, b, w, y, true, false);
+  if (s != TWQ_OK) return s;
+  if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000) return TWQ_ERR_INVALID_ARG;
+  twq::GemmCall c{twq::kModeW4A4, xq, sx, b, w, y, nullptr};
+  if (!twq::pair_eligible(c)) return TWQ_ERR_UNSUPPORTED;
+  return from_cuda(twq::launch_pair_stall_selftest(c, reinterpret_cast<cudaStream_t>(stream),
+                                                   static_cast<unsigned long long>(wait_limit_ns)));
 }
 
 void twq_release_cache(void) {
@@ -357,9 +390,11 @@ int twq_launches_per_call(const char* ep) {
   if (!strcmp(ep, "twq_fused_linear") || !strcmp(ep, "twq_w4a4_only") ||
       !strcmp(ep, "twq_lowrank_only") || !strcmp(ep, "twq_fused_linear_x") ||
       !strcmp(ep, "twq_fused_linear_x_host") || !strcmp(ep, "twq_fused_linear_a8") ||
-      !strcmp(ep, "twq_fused_linear_x_a8"))
+      !strcmp(ep, "twq_fused_linear_x_a8") || !strcmp(ep, "twq_quantize_act_i8") ||
+      !strcmp(ep, "twq_fused_linear_i8"))
     return 1;
-  if (!strcmp(ep, "twq_linear_host")) return 2;  // 1 for the batches twq_fused_linear_x takes
+  if (!strcmp(ep, "twq_linear_host")) return 2;
+  if (!strcmp(ep, "twq_selftest_wait_timeout")) return 1;  // 1 for the batches twq_fused_linear_x takes
   if (!strcmp(ep, "twq_unfused_linear") || !strcmp(ep, "twq_unfused_linear_noalloc")) return 4;
   if (!strcmp(ep, "twq_fold_transforms")) return 5;
   return -1;

@@ -1192,6 +1192,8 @@ cudaError_t launch_mode(const GemmCall& c, cudaStream_t st) {
 cudaError_t launch_gemm(const GemmCall& c, cudaStream_t st, int* launches) {
   if (c.a8 && c.mode != kModeFused && c.mode != kModeW4A4) return cudaErrorInvalidValue;
   if (launches) ++*launches;
+  // Prefill batches of the three layer modes run on CTA pairs (256 x 256 tiles).
+  if (pair_eligible(c)) return launch_pair(c, st);
   switch (c.mode) {
     case kModeFused:
       return c.a8 ? launch_mode<kModeFused, 128, true>(c, st) : launch_mode<kModeFused, 128>(c, st);

@@ -29,22 +29,37 @@ struct GemmCall {
   const uint16_t* h_global; // kModeS2F32 only: bf16 H, b x r
   const uint16_t* x = nullptr;  // decode kernel only: BF16 X, quantized in the kernel
   int64_t ldx = 0;
-  bool a8 = false;  // W4A8: xq holds int8 codes (q_max = 127), b x m
+  bool a8 = false;  // xq holds one int8 code per element, b x m (W4A8's 8-bit codes, or
+                    // 4-bit codes stored in bytes)
   const uint8_t* l2q = nullptr;  // kModeFusedS2Q: L2 as 4-bit codes, n x r/2 (K-major)
   const float* sl2q = nullptr;   // kModeFusedS2Q: their scales, (r/128) x n
 };
 
 // Host-side launchers; all return cudaSuccess or the launch error.
 cudaError_t launch_gemm(const GemmCall& call, cudaStream_t stream, int* launches);
-// a8: int8 codes with q_max = 127 (b x m bytes), else packed nibbles (b x m/2 bytes).
+// a8: int8 codes with q_max = 127 (b x m bytes); bytes4: 4-bit codes (q_max = 7) one
+// per byte (b x m bytes); else packed nibbles (b x m/2 bytes).
 cudaError_t launch_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
-                                float* sx, cudaStream_t stream, bool a8 = false);
+                                float* sx, cudaStream_t stream, bool a8 = false,
+                                bool bytes4 = false);
 cudaError_t launch_pack_cols(const uint16_t* w, int64_t m, int64_t cols, uint8_t* q, float* s,
                              cudaStream_t stream);
 cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out,
                                   cudaStream_t stream);
 cudaError_t launch_add_cast(const float* a, const float* b, int64_t count, uint16_t* y,
                             cudaStream_t stream);
+
+// Prefill kernel on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2): the fused,
+// W4A4-only and low-rank-only layers with 4-bit X codes, n % 256 == 0, m >= 256,
+// b > 16.
+bool pair_eligible(const GemmCall& call);
+cudaError_t launch_pair(const GemmCall& call, cudaStream_t stream);
+// Self-test of the bounded waits: the kernel with its X copies withheld and the
+// given wait limit, so that every wait on X runs out and the kernel leaves through
+// its abort path (status site codes 41-52 in the pair status word).
+cudaError_t launch_pair_stall_selftest(const GemmCall& call, cudaStream_t stream,
+                                       unsigned long long wait_ns);
+cudaError_t read_and_clear_pair_status(int* code);
 
 // Decode-shape kernel (b <= 16, split K over a 4- or 8-CTA cluster).
 bool decode_eligible(const GemmCall& call);

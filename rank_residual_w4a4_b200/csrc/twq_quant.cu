@@ -16,9 +16,9 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as
 
 // One half-warp per (token, group): lane l of the half covers elements
 // [8l, 8l + 8) of the group; a warp covers two consecutive groups of one row.
-// kA8: q_max = 127, one int8 code per element (W4A8 activations); else q_max = 7,
-// two nibbles per byte.
-template <bool kA8>
+// kQmax: 7 (4-bit codes) or 127 (W4A8's 8-bit codes). kBytes: one int8 code per
+// element (element k of a row in byte k); else two's-complement nibbles, two per byte.
+template <int kQmax, bool kBytes>
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x,
                                                            int64_t b, int m, int64_t ldx,
                                                            uint8_t* __restrict__ xq,
@@ -51,13 +51,17 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
   for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(f[k]));
 #pragma unroll
   for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-  constexpr int kQmax = kA8 ? 127 : 7;
   const Eq1Scale ks = eq1_scale<kQmax>(a);
   const float s = ks.s;
   uint32_t code[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (s != 0.0f) eq1_codes<kQmax>(f, ks, code);
   if (valid) {
-    if constexpr (kA8) {  // element 8l + k in byte k
+    if constexpr (kBytes) {  // element 8l + k in byte k, as a two's-complement int8
+      if constexpr (kQmax == 7) {  // the codes are 4-bit: sign-extend them to 8 bits
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          code[k] = static_cast<uint32_t>(static_cast<int32_t>(code[k] << 28) >> 28) & 0xFFu;
+      }
       const uint2 v = make_uint2(code[0] | (code[1] << 8) | (code[2] << 16) | (code[3] << 24),
                                  code[4] | (code[5] << 8) | (code[6] << 16) | (code[7] << 24));
       *reinterpret_cast<uint2*>(xq + row * m + g * 128 + l * 8) = v;
@@ -139,15 +143,18 @@ __global__ void add_cast_kernel(const float4* __restrict__ a, const float4* __re
 }  // namespace
 
 cudaError_t launch_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
-                                float* sx, cudaStream_t st, bool a8) {
+                                float* sx, cudaStream_t st, bool a8, bool bytes4) {
   const int G = static_cast<int>(m / 128);
   const int64_t warps = b * ((G + 1) / 2);
   const int64_t blocks = (warps + 7) / 8;
   if (a8)
-    quantize_act_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+    quantize_act_kernel<127, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        x, b, static_cast<int>(m), ldx, xq, sx);
+  else if (bytes4)
+    quantize_act_kernel<7, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
         x, b, static_cast<int>(m), ldx, xq, sx);
   else
-    quantize_act_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+    quantize_act_kernel<7, false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
         x, b, static_cast<int>(m), ldx, xq, sx);
   return cudaGetLastError();
 }

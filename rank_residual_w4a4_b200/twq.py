@@ -30,7 +30,8 @@ EXPORTS = ("twq_version", "twq_status_string", "twq_weights_sizes", "twq_act_siz
            "twq_fused_linear_x", "twq_fold_workspace_bytes", "twq_fold_transforms",
            "twq_fused_linear_x_host", "twq_quantize_act_a8", "twq_fused_linear_a8",
            "twq_fused_linear_x_a8", "twq_pack_l2_int4", "twq_fused_linear_s2q",
-           "twq_linear_host", "twq_release_cache")
+           "twq_linear_host", "twq_release_cache", "twq_selftest_wait_timeout",
+           "twq_quantize_act_i8", "twq_fused_linear_i8")
 
 
 class TwqError(RuntimeError):
@@ -84,6 +85,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twq_fold_transforms": ([P, P, P, P, P, I, I, I, P, P, P, P, S, P], ctypes.c_int),
         "twq_linear_host": ([P, I, P, P, P, P, P, P, P], ctypes.c_int),
         "twq_release_cache": ([], None),
+        "twq_selftest_wait_timeout": ([P, P, I, P, P, I, P], ctypes.c_int),
+        "twq_quantize_act_i8": ([P, I, I, I, P, P, P], ctypes.c_int),
+        "twq_fused_linear_i8": ([P, P, I, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -227,6 +231,33 @@ def quantize_act_a8(x: torch.Tensor, xq8: torch.Tensor | None = None,
     return xq8, sx
 
 
+def quantize_act_i8(x: torch.Tensor, xq8: torch.Tensor | None = None,
+                    sx: torch.Tensor | None = None, stream=None):
+    """BF16 X (b x m) -> the 4-bit codes of quantize_act stored one per byte (b x m int8,
+    values in [-7, 7]) and the same scales (b x m/128 fp32)."""
+    b, m = x.shape
+    if xq8 is None:
+        xq8 = torch.empty((b, m), dtype=torch.int8, device=x.device)
+    if sx is None:
+        sx = torch.empty((b, max(m // 128, 1)), dtype=torch.float32, device=x.device)
+    _check(load().twq_quantize_act_i8(_dev(x, "x", torch.bfloat16), b, m, m,
+                                      _dev(xq8, "xq8", torch.int8), _dev(sx, "sx", torch.float32),
+                                      _stream(stream)), "twq_quantize_act_i8")
+    return xq8, sx
+
+
+def fused_linear_i8(xq8, sx, w: Weights, y=None, stream=None):
+    """The fused layer on activation codes stored one per byte (quantize_act_i8)."""
+    b = xq8.shape[0]
+    if y is None:
+        y = torch.empty((b, w.n), dtype=torch.bfloat16, device=xq8.device)
+    cw = w.c_struct()
+    _check(load().twq_fused_linear_i8(_dev(xq8, "xq8", torch.int8), _dev(sx, "sx", torch.float32),
+                                      b, ctypes.byref(cw), _dev(y, "y", torch.bfloat16),
+                                      _stream(stream)), "twq_fused_linear_i8")
+    return y
+
+
 def fused_linear_a8(xq8, sx, w: Weights, y=None, stream=None):
     """The fused W4A8 layer on codes from quantize_act_a8 (decode batches, b <= 16)."""
     b = xq8.shape[0]
@@ -354,7 +385,7 @@ class LinearHostStep:
     def __init__(self, b: int, m: int, n: int, device, stream=None, y_host: torch.Tensor | None = None):
         self._b, self._m, self._n = b, m, n
         self.x_dev = torch.empty((b, m), dtype=torch.bfloat16, device=device)
-        self.xq = torch.empty((b, m // 2), dtype=torch.uint8, device=device)
+        self.xq = torch.empty((b, m), dtype=torch.int8, device=device)  # codes, one per byte
         self.sx = torch.empty((b, max(m // 128, 1)), dtype=torch.float32, device=device)
         self.y_dev = torch.empty((b, n), dtype=torch.bfloat16, device=device)
         if y_host is None:
@@ -377,6 +408,23 @@ class LinearHostStep:
         _check(self._fn(x_host.data_ptr(), self._b, ctypes.byref(w.c_struct()), xd, xq, sx, yd,
                         yh, self._st), "twq_linear_host")
         return self.y_host
+
+
+def selftest_wait_timeout(xq, sx, w: Weights, y=None, wait_limit_ns: int = 100000, stream=None):
+    """Run the prefill kernel with its X copies withheld and short bounded waits (see
+    twq_selftest_wait_timeout); returns y (unspecified). Read device_status() after it."""
+    return _layer_extra("twq_selftest_wait_timeout", xq, sx, w, y, stream, int(wait_limit_ns))
+
+
+def _layer_extra(fn: str, xq, sx, w: Weights, y, stream, extra):
+    b = xq.shape[0]
+    if y is None:
+        y = torch.empty((b, w.n), dtype=torch.bfloat16, device=xq.device)
+    cw = w.c_struct()
+    _check(getattr(load(), fn)(_dev(xq, "xq", torch.uint8), _dev(sx, "sx", torch.float32), b,
+                               ctypes.byref(cw), _dev(y, "y", torch.bfloat16), extra,
+                               _stream(stream)), fn)
+    return y
 
 
 def release_cache() -> None:

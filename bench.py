@@ -101,7 +101,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     # the files a capture of each kernel depends on
     "decode": ("twq_decode_sm100.cu", "sm100_ptx.cuh", "twq_eq1.cuh"),
-    "gemm": ("twq_gemm_sm100.cu", "sm100_ptx.cuh"),
+    "pair": ("twq_pair_sm100.cu", "sm100_ptx.cuh"),
 }
 
 
@@ -114,7 +114,8 @@ def kernel_source_hash(kind):
 
 
 def kernel_kind(workload):
-    return "decode" if describe(workload.replace("_x", ""))[1] <= 16 else "gemm"
+    # prefill batches of the workloads here all run on the CTA-pair kernel
+    return "decode" if describe(workload.replace("_x", ""))[1] <= 16 else "pair"
 
 
 def profiled_traffic(workload):

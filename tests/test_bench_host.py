@@ -40,7 +40,8 @@ def test_traffic_table_is_tied_to_the_kernel_sources():
         h = bench.kernel_source_hash(bench.kernel_kind(wl))
         got = bench.profiled_traffic(wl)
         assert got == (int(nbytes) if hh == h else None)
-    assert bench.kernel_kind("decode16_x") == "decode" and bench.kernel_kind("gateup") == "gemm"
+    assert bench.kernel_kind("decode16_x") == "decode" and bench.kernel_kind("gateup") == "pair"
+    assert bench.profiled_traffic("large") is not None  # captured from the committed sources
 
 
 def _rank_main(rank, world, port, out):

@@ -76,11 +76,11 @@ __device__ __forceinline__ uint32_t eq1_bits(float t) {
 __device__ __forceinline__ uint32_t eq1_nibble(float t) { return eq1_bits<0xFu>(t); }
 
 // Codes of N values of one group (needs k.s > 0), as two's-complement nibbles
-// (q_max = 7) or bytes (q_max = 127); branch-free for fast scales.
-template <int QMAX, int N>
+// (q_max = 7) or bytes (q_max = 127, or kMask = 0xFF: the 4-bit codes sign-extended
+// to int8, which the same low bits give); branch-free for fast scales.
+template <int QMAX, int N, uint32_t kMask = (QMAX == 7 ? 0xFu : 0xFFu)>
 __device__ __forceinline__ void eq1_codes(const float (&v)[N], const Eq1Scale& k,
                                           uint32_t (&code)[N]) {
-  constexpr uint32_t kMask = QMAX == 7 ? 0xFu : 0xFFu;
   if (k.fast) {
 #pragma unroll
     for (int i = 0; i < N; ++i) {

@@ -15,9 +15,12 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as
 
 
 // One half-warp per (token, group): lane l of the half covers elements
-// [8l, 8l + 8) of the group; a warp covers two consecutive groups of one row.
-// kQmax: 7 (4-bit codes) or 127 (W4A8's 8-bit codes). kBytes: one int8 code per
-// element (element k of a row in byte k); else two's-complement nibbles, two per byte.
+// [8l, 8l + 8) of the group; a warp covers two consecutive groups of one row (a work
+// item) and takes kItems consecutive items, whose loads it issues together so each
+// thread keeps 64 bytes in flight (one 16-byte load per thread does not cover HBM
+// latency). kQmax: 7 (4-bit codes) or 127 (W4A8's 8-bit codes). kBytes: one int8 code
+// per element (element k of a row in byte k); else two's-complement nibbles, two per byte.
+constexpr int kItems = 4;
 template <int kQmax, bool kBytes>
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x,
                                                            int64_t b, int m, int64_t ldx,
@@ -28,50 +31,76 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
   pdl_launch_dependents();
   const int G = m / 128;
   const int pairs = (G + 1) / 2;
-  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t items = b * pairs;
+  const int64_t w0 = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * kItems;
   const int lane = threadIdx.x & 31;
-  const int64_t row = gw / pairs;
-  if (row >= b) return;
-  const int g = static_cast<int>(gw % pairs) * 2 + (lane >> 4);
-  const bool valid = g < G;
   const int l = lane & 15;
-  uint4 raw = make_uint4(0, 0, 0, 0);
-  if (valid) raw = __ldg(reinterpret_cast<const uint4*>(x + row * ldx + g * 128 + l * 8));
-  float f[8];
-  f[0] = bf16_bits_to_f32(raw.x & 0xFFFFu);
-  f[1] = bf16_bits_to_f32(raw.x >> 16);
-  f[2] = bf16_bits_to_f32(raw.y & 0xFFFFu);
-  f[3] = bf16_bits_to_f32(raw.y >> 16);
-  f[4] = bf16_bits_to_f32(raw.z & 0xFFFFu);
-  f[5] = bf16_bits_to_f32(raw.z >> 16);
-  f[6] = bf16_bits_to_f32(raw.w & 0xFFFFu);
-  f[7] = bf16_bits_to_f32(raw.w >> 16);
-  float a = 0.0f;
+  // item w0 + u is pair p of row `row`: one division per warp, then increments
+  int64_t row0 = w0 / pairs;
+  const int p0 = static_cast<int>(w0 - row0 * pairs);
+  int64_t rows[kItems];
+  int gs[kItems];
+  {
+    int64_t rr = row0;
+    int p = p0;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(f[k]));
-#pragma unroll
-  for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-  const Eq1Scale ks = eq1_scale<kQmax>(a);
-  const float s = ks.s;
-  uint32_t code[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  if (s != 0.0f) eq1_codes<kQmax>(f, ks, code);
-  if (valid) {
-    if constexpr (kBytes) {  // element 8l + k in byte k, as a two's-complement int8
-      if constexpr (kQmax == 7) {  // the codes are 4-bit: sign-extend them to 8 bits
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          code[k] = static_cast<uint32_t>(static_cast<int32_t>(code[k] << 28) >> 28) & 0xFFu;
+    for (int u = 0; u < kItems; ++u) {
+      rows[u] = rr;
+      gs[u] = p * 2 + (lane >> 4);
+      if (++p == pairs) {
+        p = 0;
+        ++rr;
       }
-      const uint2 v = make_uint2(code[0] | (code[1] << 8) | (code[2] << 16) | (code[3] << 24),
-                                 code[4] | (code[5] << 8) | (code[6] << 16) | (code[7] << 24));
-      *reinterpret_cast<uint2*>(xq + row * m + g * 128 + l * 8) = v;
-    } else {  // element 8l + k in nibble k (element 2p in the low nibble of byte p)
-      uint32_t word = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) word |= code[k] << (4 * k);
-      *reinterpret_cast<uint32_t*>(xq + row * (m / 2) + g * 64 + l * 4) = word;
     }
-    if (l == 0) sx[row * G + g] = s;
+  }
+  uint4 raw[kItems];
+#pragma unroll
+  for (int u = 0; u < kItems; ++u) {
+    raw[u] = make_uint4(0, 0, 0, 0);
+    if (w0 + u < items && gs[u] < G)
+      raw[u] = __ldg(reinterpret_cast<const uint4*>(x + rows[u] * ldx + gs[u] * 128 + l * 8));
+  }
+#pragma unroll
+  for (int u = 0; u < kItems; ++u) {
+    if (w0 + u >= items) break;  // the same for the whole warp
+    const int64_t row = rows[u];
+    const int g = gs[u];
+    const bool valid = g < G;
+    // BF16 -> fp32: the 16 bits become the high half
+    float f[8];
+    f[0] = __uint_as_float(__byte_perm(raw[u].x, 0u, 0x1044));
+    f[1] = __uint_as_float(raw[u].x & 0xFFFF0000u);
+    f[2] = __uint_as_float(__byte_perm(raw[u].y, 0u, 0x1044));
+    f[3] = __uint_as_float(raw[u].y & 0xFFFF0000u);
+    f[4] = __uint_as_float(__byte_perm(raw[u].z, 0u, 0x1044));
+    f[5] = __uint_as_float(raw[u].z & 0xFFFF0000u);
+    f[6] = __uint_as_float(__byte_perm(raw[u].w, 0u, 0x1044));
+    f[7] = __uint_as_float(raw[u].w & 0xFFFF0000u);
+    float a = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a = fmaxf(a, fabsf(f[k]));
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+    const Eq1Scale ks = eq1_scale<kQmax>(a);
+    const float s = ks.s;
+    uint32_t code[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (valid) {
+      if constexpr (kBytes) {  // element 8l + k in byte k, as a two's-complement int8
+        if (s != 0.0f) eq1_codes<kQmax, 8, 0xFFu>(f, ks, code);
+        const uint2 v = make_uint2(__byte_perm(__byte_perm(code[0], code[1], 0x0040),
+                                               __byte_perm(code[2], code[3], 0x0040), 0x5410),
+                                   __byte_perm(__byte_perm(code[4], code[5], 0x0040),
+                                               __byte_perm(code[6], code[7], 0x0040), 0x5410));
+        *reinterpret_cast<uint2*>(xq + row * m + g * 128 + l * 8) = v;
+      } else {  // element 8l + k in nibble k (element 2p in the low nibble of byte p)
+        if (s != 0.0f) eq1_codes<kQmax>(f, ks, code);
+        uint32_t word = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) word |= code[k] << (4 * k);
+        *reinterpret_cast<uint32_t*>(xq + row * (m / 2) + g * 64 + l * 4) = word;
+      }
+      if (l == 0) sx[row * G + g] = s;
+    }
   }
 }
 
@@ -145,7 +174,7 @@ __global__ void add_cast_kernel(const float4* __restrict__ a, const float4* __re
 cudaError_t launch_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
                                 float* sx, cudaStream_t st, bool a8, bool bytes4) {
   const int G = static_cast<int>(m / 128);
-  const int64_t warps = b * ((G + 1) / 2);
+  const int64_t warps = (b * ((G + 1) / 2) + kItems - 1) / kItems;
   const int64_t blocks = (warps + 7) / 8;
   if (a8)
     quantize_act_kernel<127, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(

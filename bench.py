@@ -954,8 +954,13 @@ def run_profile(args):
     twq.load()
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    prob = Problem(args.workload, device, copies=1)
     kind = args.profile
+    if kind == "fold":  # the offline transform fold at the decode layer's dimensions
+        res = fold_entry(device, reps=max(1, args.steps))
+        print(json.dumps({"profile": kind, "fold_ms": res["fold_ms"],
+                          "device_status": twq.device_status()}), flush=True)
+        return
+    prob = Problem(args.workload, device, copies=1)
     b, m = prob.b, prob.m
     w, x, xq, sx, y = prob.weights[0], prob.x[0], prob.xq[0], prob.sx[0], prob.y[0]
     twq.quantize_act(x, xq, sx)
@@ -1008,7 +1013,7 @@ def main():
     ap.add_argument("--clock-seconds", type=float, default=1.0,
                     help="seconds of warm-up replays before the timed region (clock sampling)")
     ap.add_argument("--profile", choices=["step", "quant", "quant_i8", "fused", "fused_i8", "w4a4",
-                                          "lowrank", "fused_x", "a8", "s2q", "unfused"],
+                                          "lowrank", "fused_x", "a8", "s2q", "unfused", "fold"],
                     help="plain run for a profiler: W + K eager calls of one entry point on one "
                          "copy of the inputs, no timing")
     args = ap.parse_args()

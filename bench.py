@@ -7,8 +7,10 @@ One step is one pass of the hot path over one batch on inputs already resident
 in HBM: BF16 X to BF16 Y through the online activation quantizer and the fused
 dual-component layer. For decode batches (b <= 16) that is one launch of
 twq_fused_linear_x, which quantizes X inside the layer kernel; otherwise it is
-twq_quantize_act followed by twq_fused_linear (the two-call step is timed for
-decode batches too and reported beside it). Steps run from a CUDA
+twq_quantize_act_i8 followed by twq_fused_linear_i8 (the 4-bit codes stored one
+per byte). The step on packed codes (twq_quantize_act + twq_fused_linear) is timed
+beside it. The default workload is the large MLP layer (b = 8192, m = 5120,
+n = 25600, r = 256), the largest that fits one GPU. Steps run from a CUDA
 graph on one stream; the K timed steps are bracketed by a barrier and a device
 synchronize, timed with CUDA events, max over ranks. Packed weights rotate over
 enough copies that consecutive uses of one copy are more than 2x the 126 MB L2
@@ -602,7 +604,8 @@ def run_e2e(prob, K, W, world, device):
         calls = [twq.LinearHostStep(r1 - r0, prob.m, prob.n, device,
                                     stream=streams[k % nstreams], y_host=yh[r0:r1])
                  for k, (r0, r1) in enumerate(chunks)]
-        path = ("twq_linear_host (H2D, twq_quantize_act, twq_fused_linear, D2H in one C-ABI call) "
+        path = ("twq_linear_host (H2D, the quantizer to codes one per byte, the layer on them, D2H, "
+                "in one C-ABI call) "
                 "per %d-row chunk via twq.LinearHostStep, eager, four streams in rotation" % chunk)
     xparts = [xh[r0:r1] for r0, r1 in chunks]
 

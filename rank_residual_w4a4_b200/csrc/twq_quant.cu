@@ -17,11 +17,11 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as
 // One half-warp per (token, group): lane l of the half covers elements
 // [8l, 8l + 8) of the group; a warp covers two consecutive groups of one row (a work
 // item) and takes kItems consecutive items, whose loads it issues together so each
-// thread keeps 64 bytes in flight (one 16-byte load per thread does not cover HBM
-// latency). kQmax: 7 (4-bit codes) or 127 (W4A8's 8-bit codes). kBytes: one int8 code
-// per element (element k of a row in byte k); else two's-complement nibbles, two per byte.
-constexpr int kItems = 4;
-template <int kQmax, bool kBytes>
+// thread keeps 64 bytes in flight on large inputs (one 16-byte load per thread does
+// not cover HBM latency); small inputs take one item per warp, for more blocks.
+// kQmax: 7 (4-bit codes) or 127 (W4A8's 8-bit codes). kBytes: one int8 code per
+// element (element k of a row in byte k); else two's-complement nibbles, two per byte.
+template <int kQmax, bool kBytes, int kItems>
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x,
                                                            int64_t b, int m, int64_t ldx,
                                                            uint8_t* __restrict__ xq,
@@ -171,20 +171,28 @@ __global__ void add_cast_kernel(const float4* __restrict__ a, const float4* __re
 
 }  // namespace
 
+template <int kItems>
+void launch_quantize_items(const uint16_t* x, int64_t b, int m, int64_t ldx, uint8_t* xq, float* sx,
+                           cudaStream_t st, bool a8, bool bytes4) {
+  const int64_t items = b * ((m / 128 + 1) / 2);
+  const int64_t warps = (items + kItems - 1) / kItems;
+  const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+  if (a8)
+    quantize_act_kernel<127, true, kItems><<<blocks, 256, 0, st>>>(x, b, m, ldx, xq, sx);
+  else if (bytes4)
+    quantize_act_kernel<7, true, kItems><<<blocks, 256, 0, st>>>(x, b, m, ldx, xq, sx);
+  else
+    quantize_act_kernel<7, false, kItems><<<blocks, 256, 0, st>>>(x, b, m, ldx, xq, sx);
+}
+
 cudaError_t launch_quantize_act(const uint16_t* x, int64_t b, int64_t m, int64_t ldx, uint8_t* xq,
                                 float* sx, cudaStream_t st, bool a8, bool bytes4) {
-  const int G = static_cast<int>(m / 128);
-  const int64_t warps = (b * ((G + 1) / 2) + kItems - 1) / kItems;
-  const int64_t blocks = (warps + 7) / 8;
-  if (a8)
-    quantize_act_kernel<127, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        x, b, static_cast<int>(m), ldx, xq, sx);
-  else if (bytes4)
-    quantize_act_kernel<7, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        x, b, static_cast<int>(m), ldx, xq, sx);
+  // Four items per warp once there are enough of them for about 4 blocks per SM.
+  const int64_t items = b * ((m / 128 + 1) / 2);
+  if (items >= 148 * 4 * 8 * 4)
+    launch_quantize_items<4>(x, b, static_cast<int>(m), ldx, xq, sx, st, a8, bytes4);
   else
-    quantize_act_kernel<7, false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        x, b, static_cast<int>(m), ldx, xq, sx);
+    launch_quantize_items<1>(x, b, static_cast<int>(m), ldx, xq, sx, st, a8, bytes4);
   return cudaGetLastError();
 }
 

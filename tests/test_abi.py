@@ -245,3 +245,63 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises(ValueError):
         twq.quantize_act(x, torch.zeros(4, 256, dtype=torch.uint8),
                          torch.zeros(4, 4, dtype=torch.float32))
+
+
+def test_byte_code_entry_points_validation(lib):
+    # the prefill form: the 4-bit codes one per byte; every rejection before any launch
+    q = lib.twq_quantize_act_i8
+    assert q(None, 40, 512, 512, A, A, None) == 1
+    assert q(A, 40, 500, 512, A, A, None) == 1            # m % 128
+    assert q(A, 40, 512, 256, A, A, None) == 1            # ldx < m
+    assert q(A, 40, 512, 516, A, A, None) == 3            # row stride breaks 16 bytes
+    assert q(A, 40, 512, 512, A + 8, A, None) == 3
+    assert q(A, -1, 512, 512, A, A, None) == 1
+    assert q(None, 0, 512, 512, None, None, None) == 0    # b == 0: nothing to do
+    f = lib.twq_fused_linear_i8
+    w = _w()
+    assert f(None, A, 40, ctypes.byref(w), A, None) == 1
+    assert f(A, A, 40, None, A, None) == 1
+    assert f(A + 8, A, 40, ctypes.byref(w), A, None) == 3
+    assert f(A, A, 40, ctypes.byref(w), A + 4, None) == 3
+    assert f(A, A, 40, ctypes.byref(_w(m=500)), A, None) == 1
+    assert f(A, A, 40, ctypes.byref(_w(r=272)), A, None) == 2
+    assert f(A, A, 0, ctypes.byref(w), None, None) == 0
+
+
+def test_linear_host_validation(lib):
+    # (x_host, b, w, x_dev, xq, sx, y_dev, y_host, stream): rejections before any copy
+    f = lib.twq_linear_host
+    w = _w()
+    assert f(A, 40, None, A, A, A, A, A, None) == 1          # no weights
+    assert f(None, 40, ctypes.byref(w), A, A, A, A, A, None) == 1   # no host X
+    assert f(A, 40, ctypes.byref(w), A, A, A, A, None, None) == 1   # no host Y
+    assert f(A, 40, ctypes.byref(w), None, A, A, A, A, None) == 1   # no device X
+    assert f(A, 40, ctypes.byref(w), A, A, A, None, A, None) == 1   # no device Y
+    assert f(A, -1, ctypes.byref(w), A, A, A, A, A, None) == 1
+    assert f(None, 0, ctypes.byref(w), None, None, None, None, None, None) == 0
+    assert f(A, 40, ctypes.byref(w), A + 2, A, A, A, A, None) == 3  # misaligned device X
+    # a prefill batch needs the code and scale buffers, aligned
+    assert f(A, 40, ctypes.byref(w), A, None, A, A, A, None) == 1
+    assert f(A, 40, ctypes.byref(w), A, A, None, A, A, None) == 1
+    assert f(A, 40, ctypes.byref(w), A, A + 8, A, A, A, None) == 3
+    assert f(A, 40, ctypes.byref(w), A, A, A, A + 4, A, None) == 3
+    assert f(A, 40, ctypes.byref(_w(m=500)), A, A, A, A, A, None) == 1
+    assert f(A, 40, ctypes.byref(_w(r=272)), A, A, A, A, A, None) == 2
+
+
+def test_wait_selftest_validation(lib):
+    f = lib.twq_selftest_wait_timeout
+    w = _w(r=0)
+    assert f(None, A, 300, ctypes.byref(w), A, 100000, None) == 1
+    assert f(A + 8, A, 300, ctypes.byref(w), A, 100000, None) == 3
+    assert f(A, A, 300, ctypes.byref(w), A, 999, None) == 1            # below 1 us
+    assert f(A, A, 300, ctypes.byref(w), A, 2000000000, None) == 1     # above 1 s
+    # shapes the prefill kernel does not take are refused, nothing launched
+    assert f(A, A, 4, ctypes.byref(w), A, 100000, None) == 2           # b <= 16
+    assert f(A, A, 300, ctypes.byref(_w(n=384, r=0)), A, 100000, None) == 2  # n % 256
+
+
+def test_release_cache_is_host_only(lib):
+    # no GPU here: the call only clears host-side tables
+    lib.twq_release_cache()
+    lib.twq_release_cache()

@@ -306,16 +306,23 @@ def test_degenerate_inputs(twq, device):
 
 # --------------------------------------------------- the five workloads, full size
 
-def _full(twq, device, name, b, rows):
+def _full(twq, device, name, b, rows, byte_codes=False):
     wl = synth.WORKLOADS[name]
     x = synth.make_x(wl, b=b)
     R, L1, L2 = synth.make_weights(wl)
     w = _pack(twq, device, R, L1, L2)
-    xq, sx = twq.quantize_act(to_dev(x, device))
+    xd = to_dev(x, device)
+    xq, sx = twq.quantize_act(xd)
     y = bits_of(twq.fused_linear(xq, sx, w))
     rows = np.arange(b) if rows is None else rows
     ref = _oracle_y(x, R, L1, L2, oracle.FUSED, rows=rows)
     assert_y_close(y[rows], ref, "%s b=%d" % (name, b))
+    if byte_codes:
+        # the benchmark's step: the same codes one per byte, the layer on them; the whole Y
+        # is bitwise that of the packed path checked above
+        xq8, sx8 = twq.quantize_act_i8(xd)
+        assert np.array_equal(sx8.cpu().numpy().view(np.uint32), sx.cpu().numpy().view(np.uint32))
+        assert np.array_equal(bits_of(twq.fused_linear_i8(xq8, sx8, w)), y)
     _status_clean(twq)
     return y, rows
 
@@ -328,6 +335,7 @@ def test_workload_all_rows(twq, device, name, b):
 @pytest.mark.parametrize("name", ["gateup", "down", "large"])
 def test_workload_rows_of_every_row_block(twq, device, name):
     """Full-size prefill workloads: two seeded rows of every 128-row block (every row
-    block of the persistent schedule, so every CTA's work), all columns."""
+    block of the persistent schedule, so every CTA's work), all columns; and the byte-code
+    path the benchmark times, bitwise against the whole packed-code Y."""
     wl = synth.WORKLOADS[name]
-    _full(twq, device, name, wl.b, block_rows(wl.b, per_block=2, seed=11))
+    _full(twq, device, name, wl.b, block_rows(wl.b, per_block=2, seed=11), byte_codes=True)

@@ -62,6 +62,7 @@ constexpr int kThreads = 512;
 constexpr int kSS = 4;     // weight-scale slots, four K groups each (the weight producer
                            // loads them, so a deep ring keeps it ahead of the drain)
 constexpr int kMaxR = 256;
+constexpr int kMaxPairs = 128;  // runs in the launch's tile partition
 
 // Wait sites of this kernel (recorded in g_pair_status).
 enum PairSite : int {
@@ -100,6 +101,7 @@ struct PairArgs {
   int64_t b;
   int m, n, r, G;
   int col_tiles, num_items;  // pair tiles of 256 x 256
+  int bounds[kMaxPairs + 1];  // pair p takes tiles [bounds[p], bounds[p + 1]) in row-block-major order
   unsigned long long wait_ns;
   int stall;  // self-test: no copy of X is issued, so every wait on X runs out
 };
@@ -377,8 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int pair = static_cast<int>(blockIdx.x) >> 1;
   const int pairs = static_cast<int>(gridDim.x) >> 1;
-  const int t_begin = static_cast<int>((int64_t)pair * args.num_items / pairs);
-  const int t_end = static_cast<int>((int64_t)(pair + 1) * args.num_items / pairs);
+  const int t_begin = args.bounds[pair];
+  const int t_end = args.bounds[pair + 1];
+  (void)pairs;
   const int row_half = static_cast<int>(rank) * 128;  // this CTA's rows / columns in the pair tile
 
   if (warp < 8) {
@@ -848,6 +851,46 @@ int resident_pairs_of() {
   return cache[dev];
 }
 
+// Contiguous runs of tiles (row-block-major) for `pairs` pairs that minimize the largest
+// run's cost in K-group steps: each tile costs its residual groups plus about one step of
+// stage 2 and epilogue, and a run pays a stage-1 pass (G steps, cheaper when r <= 128)
+// at its start and at every row-block change. An equal split of the tiles can leave
+// the slowest pair with two stage-1 passes; when a layer has few tiles per pair (the
+// down projection: 3.5) that pass is as large as a tile. Binary search on the cost
+// bound with a greedy fill, which is optimal for contiguous runs of positive costs.
+void partition_items(int num_items, int col_tiles, int G, bool res, bool h, int r, int pairs,
+                     int* bounds) {
+  const int64_t tile = 10 * ((res ? G : 0) + 1);
+  const int64_t hpass = h ? (r <= 128 ? 6 : 10) * static_cast<int64_t>(G) : 0;
+  auto runs_for = [&](int64_t cap, int* out) {
+    int runs = 0;
+    int64_t cost = 0;
+    int start = 0;
+    for (int t = 0; t < num_items; ++t) {
+      const bool new_rb = t > start && t / col_tiles != (t - 1) / col_tiles;
+      int64_t add = tile + (new_rb ? hpass : 0);
+      if (t == start) add = tile + hpass;
+      if (t > start && cost + add > cap) {
+        if (out) out[runs] = start;
+        ++runs;
+        start = t;
+        cost = tile + hpass;
+      } else {
+        cost += add;
+      }
+    }
+    if (out) out[runs] = start;
+    return runs + 1;
+  };
+  int64_t lo = tile + hpass, hi = (tile + hpass) * static_cast<int64_t>(num_items);
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if (runs_for(mid, nullptr) <= pairs) hi = mid; else lo = mid + 1;
+  }
+  const int used = runs_for(lo, bounds);
+  for (int p = used; p <= pairs; ++p) bounds[p] = num_items;  // the rest get no tiles
+}
+
 template <int kMode, bool kXB>
 cudaError_t launch_pair_mode(const GemmCall& c, cudaStream_t st, unsigned long long wait_ns,
                              int stall) {
@@ -893,7 +936,8 @@ cudaError_t launch_pair_mode(const GemmCall& c, cudaStream_t st, unsigned long l
   if (e != cudaSuccess) return e;
   const int rp = resident_pairs_of<kMode, kXB>();
   if (rp <= 0) return cudaErrorInvalidConfiguration;
-  const int pairs = std::min(rp, a.num_items);
+  const int pairs = std::min(std::min(rp, a.num_items), kMaxPairs);
+  partition_items(a.num_items, a.col_tiles, a.G, T::res, T::h, a.r, pairs, a.bounds);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

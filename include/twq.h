@@ -300,9 +300,10 @@ TWQ_API twq_status twq_fused_linear_x_a8(const uint16_t* x, int64_t ldx, int64_t
  *   l2t is not read); l2q, sl2q from twq_pack_l2_int4; y b x n BF16. One launch; H
  *   never leaves the chip. Decode batches (b <= 16, r == 128, m <= 8192) run the
  *   split-K decode kernel, whose CTAs exchange per-token maxima of H over the
- *   cluster; other shapes run the tensor-core GEMM kernel, where H's codes overwrite
- *   it in shared memory and feed r/128 more int8 K groups of the residual
- *   accumulation. Errors as twq_fused_linear; r outside {128, 256} returns
+ *   cluster; other shapes run the tensor-core prefill kernel (on CTA pairs when
+ *   b > 16, m >= 256 and n % 256 == 0, else on single CTAs), where H's codes
+ *   overwrite it in shared memory and feed r/128 more int8 K groups of the
+ *   residual accumulation. Errors as twq_fused_linear; r outside {128, 256} returns
  *   TWQ_ERR_UNSUPPORTED (r == 0: TWQ_ERR_INVALID_ARG).
  */
 TWQ_API twq_status twq_pack_l2_int4(const uint16_t* L2, int64_t r, int64_t n, uint8_t* l2q,

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libtwq.so")
 SOURCES = ["twq_api.cu", "twq_gemm_sm100.cu", "twq_pair_sm100.cu", "twq_decode_sm100.cu",
            "twq_quant.cu", "twq_noalloc.cu", "twq_fold.cu"]
-HEADERS = ["sm100_ptx.cuh", "twq_internal.h", "twq_eq1.cuh"]
+HEADERS = ["sm100_ptx.cuh", "twq_internal.h", "twq_eq1.cuh", "twq_hrequant.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

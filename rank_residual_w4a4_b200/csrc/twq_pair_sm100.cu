@@ -13,6 +13,9 @@
 //     reuse (H never goes to HBM);
 //   * residual: Y_res = sum_g sx[i,g] sr[g,j] (Q(X)_g Q(R)_g), same scheme (N = 256);
 //   * stage 2: Y_lr = bf16(H) L2 with kind::f16 MMAs, fp32 accumulation in tensor memory;
+//     or, in the INT4 stage-2 mode (§4.3 item 2), bf16(H) requantized on chip per token and
+//     group of 128 along r (Eq. (1)), and Q_H Q(V) run as r/128 more int8 K groups of the
+//     residual accumulation (scales s_H per token, s_V per column);
 //   * one epilogue: Y = bf16(Y_res + Y_lr), a single store.
 // The weight codes are unpacked to 16 q (two logic operations per four bytes). X
 // arrives in one of two forms:
@@ -50,6 +53,7 @@
 #include <mutex>
 
 #include "sm100_ptx.cuh"
+#include "twq_hrequant.cuh"
 #include "twq_internal.h"
 
 namespace twq {
@@ -68,7 +72,7 @@ constexpr int kMaxPairs = 128;  // runs in the launch's tile partition
 enum PairSite : int {
   kPSiteXEmpty = 41, kPSiteBEmpty = 42, kPSiteScaleEmpty = 43, kPSiteUnpackFull = 44,
   kPSiteUnpackEmpty = 45, kPSiteL2 = 46, kPSiteMmaFull = 47, kPSiteMmaAcc = 48, kPSiteMmaH = 49,
-  kPSiteDrainAcc = 50, kPSiteDrainScale = 51, kPSiteFinal = 52,
+  kPSiteDrainAcc = 50, kPSiteDrainScale = 51, kPSiteFinal = 52, kPSiteHq = 53,
 };
 
 // Shared memory. A packed slot holds two K groups: (unless kXB) X 128 rows x 128
@@ -88,7 +92,8 @@ struct Layout {
   static constexpr int kHBytes = 128 * kMaxR * 2;      // r/64 chunks of 128 x 64 BF16
   static constexpr int kOffScale = kOffH + kHBytes;
   static constexpr int kScaleSlot = 4 * 256 * 4;       // four groups of up to 256 columns
-  static constexpr int kOffBar = kOffScale + kSS * kScaleSlot;
+  static constexpr int kOffShq = kOffScale + kSS * kScaleSlot;  // INT4 stage 2: s_H, 128 x 2
+  static constexpr int kOffBar = kOffShq + 128 * 2 * 4;
   static constexpr int kNumBars = 40;
   static constexpr int kBytes = kOffBar + kNumBars * 8 + 32;
   static constexpr int kAlloc = kBytes + 1024;         // room to align the base to 1 KB
@@ -108,8 +113,10 @@ struct PairArgs {
 
 template <int kMode>
 struct Traits {
-  static constexpr bool res = kMode == kModeFused || kMode == kModeW4A4;
-  static constexpr bool h = kMode == kModeFused || kMode == kModeLowRank;
+  static constexpr bool s2q = kMode == kModeFusedS2Q;  // INT4 stage 2
+  static constexpr bool res = kMode == kModeFused || kMode == kModeW4A4 || s2q;
+  static constexpr bool h = kMode == kModeFused || kMode == kModeLowRank || s2q;
+  static constexpr bool s2 = h && !s2q;                // BF16 stage 2 (kind::f16)
 };
 
 struct Ring {
@@ -291,7 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     twq_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
                     const __grid_constant__ CUtensorMap tm_l1, const __grid_constant__ CUtensorMap tm_l2,
                     const __grid_constant__ CUtensorMap tm_sr,
-                    const __grid_constant__ CUtensorMap tm_sl1, const PairArgs args) {
+                    const __grid_constant__ CUtensorMap tm_sl1,
+                    const __grid_constant__ CUtensorMap tm_sv, const PairArgs args) {
   using L = Layout<kXB>;
   using T = Traits<kMode>;
   constexpr int kPS = L::kPS;
@@ -320,6 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* hready = sempty + kSS;        // (even CTA) both CTAs' BF16 H tiles are written
   uint64_t* mdone = hready + 1;           // every MMA of the pair has completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
+  uint64_t* hq = mdone + 2;               // INT4 stage 2: the 8 drain warps' H steps
+  float* shq = reinterpret_cast<float*>(smem + L::kOffShq);  // INT4 stage 2: s_H [row][group]
+  static_assert(!(kXB && T::s2q), "the INT4 stage 2 runs on packed codes");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -327,7 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int G = args.G;
   const int r = args.r;
-  const int KC = T::h ? (r + 63) / 64 : 0;
+  const int KC = T::s2 ? (r + 63) / 64 : 0;  // BF16 stage-2 chunks of 64 along r
+  const int NQ = T::s2q ? r / 128 : 0;        // INT4 stage 2: groups of 128 along r
   const int slots = (G + 1) / 2;  // packed slots per pass over the K groups
   const WaitCtx wc{&s_abort, args.wait_ns};
 
@@ -350,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(hready, 16);
     mbar_init(mdone, 1);
+    mbar_init(hq, 8);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -364,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_l2);
       tma_prefetch_desc(&tm_sl1);
     }
+    if (T::s2q) tma_prefetch_desc(&tm_sv);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, 512);
@@ -447,6 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               p.next(kPS);
             }
           }
+          if (T::s2q && ok) {  // the V groups' packed slot brings no X: complete its barrier
+            if (!(ok = wait_on(&pempty[p.idx], p.phase ^ 1u, wc, kPSiteXEmpty))) break;
+            mbar_arrive(&xfull[p.idx]);
+            p.next(kPS);
+          }
         }
       }
       if (!ok) {
@@ -493,6 +512,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.next(kPS);
           }
         }
+        if (T::s2q && ok) {
+          // INT4 stage 2: the V groups' scales s_V (rows beyond r/128 read as zeros) and
+          // this CTA's 128 columns of the 4-bit V codes, both groups in one copy (the
+          // half beyond r/2 bytes reads as zeros when r = 128)
+          if (!(ok = wait_on(&sempty[q.idx], q.phase ^ 1u, wc, kPSiteScaleEmpty))) break;
+          mbar_arrive_expect_tx(&sfull[q.idx], 256 * 4 * 4);
+          tma_load_2d(scl + q.idx * (L::kScaleSlot / 4), &tm_sv, &sfull[q.idx], it.ct * 256, 0);
+          spend |= 1u << q.idx;
+          spend_ph = (spend_ph & ~(1u << q.idx)) | (q.phase << q.idx);
+          q.next(kSS);
+          if (!(ok = wait_on(&pempty[p.idx], p.phase ^ 1u, wc, kPSiteBEmpty))) break;
+          mbar_arrive_expect_tx(&bfull[p.idx], 128 * 128);
+          tma_load_2d(pack + p.idx * L::kPack + L::kPackX, &tm_l2, &bfull[p.idx], 0,
+                      it.ct * 256 + row_half);
+          pend |= 1u << p.idx;
+          pend_ph = (pend_ph & ~(1u << p.idx)) | (p.phase << p.idx);
+          p.next(kPS);
+        }
       }
       if (!ok) {
         int never = 0;
@@ -532,7 +569,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             a.next(2);
           }
         }
-        if (T::h && ok) {
+        if (T::s2q && ok) {
+          // INT4 stage 2: Q_H Q(V), A = this row block's requantized H of group g2 (16*q
+          // codes over the group's first 16 KB of the H tile, in both CTAs)
+          if (it.need_h) {
+            if (!(ok = wait_on(hready, h_phase, wc, kPSiteMmaH))) break;
+            h_phase ^= 1u;
+          }
+          const uint32_t idesc = idesc_i8_m256(256);
+          for (int g2 = 0; g2 < NQ; ++g2) {
+            if (!(ok = wait_on(&ufull[u.idx], u.phase, wc, kPSiteMmaFull))) break;
+            if (!(ok = wait_on(&aempty[a.idx], a.phase ^ 1u, wc, kPSiteMmaAcc))) break;
+            tc_fence_after();
+            const uint32_t d = tmem + a.idx * 256;
+            const uint64_t da = smem_desc_sw128(h0 + g2 * 32768);
+            const uint64_t db = smem_desc_sw128(u0 + u.idx * L::kU + L::kUHalf);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mma_i8_pair(d, da + 2 * k, db + 2 * k, idesc, k > 0);
+            mma_commit_pair(&uempty[u.idx]);
+            mma_commit_pair(&afull[a.idx]);
+            u.next(kUS);
+            a.next(2);
+          }
+        }
+        if (T::s2 && ok) {
           // stage 2: bf16(H) (this row block's, on chip in both CTAs) x L2^T chunks
           if (it.need_h) {
             if (!(ok = wait_on(hready, h_phase, wc, kPSiteMmaH))) break;
@@ -607,7 +667,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           u.next(kUS);
         }
       }
-      if (T::h && ok) {
+      if (T::s2q && ok) {
+        // INT4 stage 2: the V groups, B only (A is the requantized H, already on chip)
+        for (int g2 = 0; g2 < NQ; ++g2) {
+          const int j = g2 & 1;
+          if (j == 0) {
+            ok = __all_sync(~0u, wait_on(&xfull[p.idx], p.phase, wc, kPSiteUnpackFull));
+            if (ok) ok = __all_sync(~0u, wait_on(&bfull[p.idx], p.phase, wc, kPSiteUnpackFull));
+            if (!ok) break;
+          }
+          if (!(ok = __all_sync(~0u, wait_on(&uempty[u.idx], u.phase ^ 1u, wc, kPSiteUnpackEmpty))))
+            break;
+          unpack_group<false>(pack + p.idx * L::kPack + L::kPackX, ustg + u.idx * L::kU + L::kUHalf,
+                              128, j, plan);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_cluster_n(ufull_lead + u.idx * 8, 1);
+            if (j == 1 || g2 == NQ - 1) mbar_arrive(&pempty[p.idx]);
+          }
+          if (j == 1 || g2 == NQ - 1) p.next(kPS);
+          u.next(kUS);
+        }
+      }
+      if (T::s2 && ok) {
         // stage 2: the L2^T chunks (this CTA's 128 columns x 64 of r, BF16, 128-byte
         // swizzle) go by TMA straight into the weight half of the unpacked slots
         for (int kc = 0; kc < KC; ++kc) {
@@ -649,6 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t hready_lead = map_peer(smem_u32(hready), 0);
     Ring a, q;
     bool ok = true;
+    uint32_t hq_phase = 0;  // INT4 stage 2: the phase of the drain warps' barrier
     float acc[128];
     for (int t = t_begin; t < t_end && ok; ++t) {
       const Item it = item_at(args, t, t_begin, T::h);
@@ -707,18 +791,56 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint4*>(hb + (col >> 6) * 16384 + sw128(row_in, (col & 63) >> 3)) = o;
             }
           }
+          if constexpr (T::s2q) {
+            // INT4 stage 2: once every drain warp's BF16 H is in the tile, thread (row, half)
+            // requantizes group `half` of its row (Eq. (1) over the group's 128 values,
+            // written back in place as 16*q codes in the 4-bit operand order, its scale to
+            // s_H); then all are done before the MMAs read the codes and the drains the
+            // scales. Both steps meet at a bounded barrier of the 8 drain warps.
+            __syncwarp();
+            if (lane == 0) mbar_arrive(hq);
+            if (!(ok = __all_sync(~0u, wait_on(hq, hq_phase, wc, kPSiteHq)))) break;
+            hq_phase ^= 1u;
+            if (half < NQ) requant_h_row(hb + half * 32768, row_in, shq + row_in * 2 + half, false, 0, 0);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(hq);
+            if (!(ok = __all_sync(~0u, wait_on(hq, hq_phase, wc, kPSiteHq)))) break;
+            hq_phase ^= 1u;
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster_n(hready_lead, 1);
         }
       }
       if (!ok) break;
+      if (T::s2q) {
+        // INT4 stage 2: group g2's accumulator (16*q by 16*q codes) scaled by s_V[col] (the
+        // scale slot) and s_H[row, g2], into the same sums as the residual
+        for (int g2 = 0; g2 < NQ; ++g2) {
+          const float shv = shq[row_in * 2 + g2];
+          if (g2 == 0)
+            if (!(ok = __all_sync(~0u, wait_on(&sfull[q.idx], q.phase, wc, kPSiteDrainScale)))) break;
+          if (!(ok = __all_sync(~0u, wait_on(&afull[a.idx], a.phase, wc, kPSiteDrainAcc)))) break;
+          tc_fence_after();
+          drain128(acc, tmem + lane_addr + a.idx * 256 + half * 128,
+                   scl + q.idx * (L::kScaleSlot / 4) + g2 * 256 + half * 128, f2_pack(shv, shv));
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_cluster_n(aempty_lead + a.idx * 8, 1);
+            if (g2 == NQ - 1) mbar_arrive(&sempty[q.idx]);
+          }
+          a.next(2);
+          if (g2 == NQ - 1) q.next(kSS);
+        }
+        if (!ok) break;
+      }
       if (!T::res) {
 #pragma unroll
         for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
       }
       // ------------------------------------------------------------ epilogue
-      if (T::h) {
+      if (T::s2) {
         if (!(ok = __all_sync(~0u, wait_on(&afull[a.idx], a.phase, wc, kPSiteDrainAcc)))) break;
         tc_fence_after();
       }
@@ -728,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 128; c += 32) {
         // Y = bf16(Y_res + Y_lr): Y_res = kDq acc (exact), Y_lr from tensor memory
         float yv[8];
-        if constexpr (T::h) {
+        if constexpr (T::s2) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_addr + a.idx * 256 + c0 + c, v);
           tmem_wait_ld();
@@ -753,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (T::h) {
+      if (T::s2) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster_n(aempty_lead + a.idx * 8, 1);
@@ -909,7 +1031,7 @@ cudaError_t launch_pair_mode(const GemmCall& c, cudaStream_t st, unsigned long l
   a.num_items = static_cast<int>((c.b + 255) / 256) * a.col_tiles;
   a.wait_ns = wait_ns;
   a.stall = stall;
-  CUtensorMap m_x{}, m_r{}, m_l1{}, m_l2{}, m_sr{}, m_sl1{};
+  CUtensorMap m_x{}, m_r{}, m_l1{}, m_l2{}, m_sr{}, m_sl1{}, m_sv{};
   const uint64_t kb = static_cast<uint64_t>(a.m / 2);
   const uint64_t G = static_cast<uint64_t>(a.G);
   constexpr CUtensorMapSwizzle kSw = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -925,10 +1047,23 @@ cudaError_t launch_pair_mode(const GemmCall& c, cudaStream_t st, unsigned long l
   }
   if (T::h) {
     ok = ok && encode(&m_l1, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->l1q, kb, a.r, kb, 128, a.r / 2, kSw);
-    ok = ok && encode(&m_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2t, a.r, a.n,
-                      static_cast<uint64_t>(a.r) * 2, 64, 128, kSw);
     ok = ok && encode(&m_sl1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->sl1, a.r, G,
                       static_cast<uint64_t>(a.r) * 4, a.r, 4, CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  if (T::s2) {
+    ok = ok && encode(&m_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2t, a.r, a.n,
+                      static_cast<uint64_t>(a.r) * 2, 64, 128, kSw);
+  }
+  if (T::s2q) {
+    // V: n columns of r/2 bytes (both groups of 128 codes in one 128-byte box; the half
+    // beyond r/2 reads as zeros when r = 128), in m_l2's place; s_V: (r/128) x n fp32,
+    // 256 columns x 4 groups per copy
+    ok = ok && c.l2q && c.sl2q &&
+         encode(&m_l2, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.l2q, static_cast<uint64_t>(a.r / 2), a.n,
+                static_cast<uint64_t>(a.r / 2), 128, 128, kSw);
+    ok = ok && encode(&m_sv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c.sl2q, a.n,
+                      static_cast<uint64_t>(a.r / 128), static_cast<uint64_t>(a.n) * 4, 256, 4,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
   }
   if (!ok) return cudaErrorInvalidValue;
   auto kern = twq_pair_kernel<kMode, kXB>;
@@ -950,7 +1085,7 @@ cudaError_t launch_pair_mode(const GemmCall& c, cudaStream_t st, unsigned long l
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, m_x, m_r, m_l1, m_l2, m_sr, m_sl1, a);
+  e = cudaLaunchKernelEx(&cfg, kern, m_x, m_r, m_l1, m_l2, m_sr, m_sl1, m_sv, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -962,6 +1097,9 @@ cudaError_t launch_pair_x(const GemmCall& c, cudaStream_t st) {
     case kModeFused: return launch_pair_mode<kModeFused, kXB>(c, st, kWaitNs, 0);
     case kModeW4A4: return launch_pair_mode<kModeW4A4, kXB>(c, st, kWaitNs, 0);
     case kModeLowRank: return launch_pair_mode<kModeLowRank, kXB>(c, st, kWaitNs, 0);
+    case kModeFusedS2Q:
+      if constexpr (!kXB) return launch_pair_mode<kModeFusedS2Q, false>(c, st, kWaitNs, 0);
+      return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }
@@ -970,11 +1108,14 @@ cudaError_t launch_pair_x(const GemmCall& c, cudaStream_t st) {
 
 bool pair_eligible(const GemmCall& c) {
   if (c.x != nullptr) return false;
-  if (c.mode != kModeFused && c.mode != kModeW4A4 && c.mode != kModeLowRank) return false;
-  if (c.a8 && c.mode == kModeLowRank) return false;
+  if (c.mode != kModeFused && c.mode != kModeW4A4 && c.mode != kModeLowRank &&
+      c.mode != kModeFusedS2Q)
+    return false;
+  if (c.a8 && (c.mode == kModeLowRank || c.mode == kModeFusedS2Q)) return false;
   const twq_weights* w = c.w;
   if (w->n % 256 != 0 || w->m < 256 || w->r > kMaxR) return false;
   if (c.mode != kModeW4A4 && w->r <= 0) return false;
+  if (c.mode == kModeFusedS2Q && (w->r % 128 != 0 || !c.l2q || !c.sl2q)) return false;
   return c.b > 16;
 }
 

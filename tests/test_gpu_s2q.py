@@ -127,6 +127,9 @@ def test_pack_l2_int4_bitexact(twq, device, r, n):
 SHAPES = [  # b, m, n, r: one and two groups of r, ragged rows, a single token, several tiles
     (5, 256, 128, 128), (16, 512, 384, 128), (129, 384, 256, 256), (300, 128, 512, 128),
     (64, 640, 128, 256), (1, 128, 128, 128), (200, 1024, 256, 256),
+    # the CTA-pair kernel (b > 16, m >= 256, n % 256 == 0): r = 128 with an odd number of K
+    # groups, ragged rows over several row blocks and column tiles, r = 256 with G odd
+    (40, 384, 512, 128), (513, 512, 768, 128), (300, 1152, 512, 256),
 ]
 
 

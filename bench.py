@@ -103,7 +103,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     # the files a capture of each kernel depends on
     "decode": ("twq_decode_sm100.cu", "sm100_ptx.cuh", "twq_eq1.cuh"),
-    "pair": ("twq_pair_sm100.cu", "sm100_ptx.cuh"),
+    "pair": ("twq_pair_sm100.cu", "sm100_ptx.cuh", "twq_hrequant.cuh", "twq_eq1.cuh"),
 }
 
 

@@ -30,17 +30,22 @@
 //                 two groups per copy);
 //   warp 1        tensor memory (both CTAs); in the even CTA, the MMA issuer;
 //   warp 2        TMA: packed 4-bit R / L1 tiles (two groups per copy) and the
-//                 per-group weight scales (four groups per copy);
+//                 per-group weight scales (four groups per copy); in the INT4 stage-2
+//                 mode also the 4-bit V codes and their scales;
 //   warp 3        kXB: TMA of X for the odd group steps (a thread issues a copy
 //                 every few hundred cycles at best, so two share the X stream);
 //   warps 4-7     unpack: 4-bit codes -> 16 q int8 in the MMA's 128-byte-swizzle
 //                 K-major layout (even codes of each 8 first in both operands, or,
 //                 with kXB, the weights in element order like the X codes);
 //                 they also bring the BF16 L2^T chunks of stage 2 by TMA;
-//   warps 8-15    drain: per-group tensor-memory loads (pipelined), fp32 scaling
-//                 and accumulation (packed f32x2 arithmetic), H -> BF16, epilogue.
+//   warps 8-15    drain: per-group tensor-memory loads of 16 columns, fp32 scaling
+//                 and accumulation (packed f32x2 arithmetic), H -> BF16 (and, in the
+//                 INT4 stage-2 mode, its requantization), epilogue.
 // The drain warps hold 128 fp32 sums per thread: their warpgroups raise their
 // register budget (setmaxnreg) and the others lower theirs.
+//
+// Each pair takes a contiguous run of tiles chosen on the host (partition_items) to
+// balance tiles against stage-1 passes.
 //
 // Every wait is bounded; a wait that runs out records its site in a device status
 // word, raises the CTA's abort flag, lets the CTA's copies in flight land, and the

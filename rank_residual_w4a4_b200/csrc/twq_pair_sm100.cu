@@ -285,6 +285,27 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// A 4 x 4 transpose of 16-byte pieces within each aligned group of four lanes: piece s
+// of lane i moves to piece i of lane s (two exchange rounds, lane distance 2 then 1).
+// The epilogue uses it so that four lanes store one row's 64 contiguous bytes.
+__device__ __forceinline__ void transpose4x4(uint32_t (&e)[4][4], int lane) {
+#pragma unroll
+  for (int m = 2; m >= 1; m >>= 1) {
+    const bool hi = (lane & m) != 0;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      if (s & m) continue;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t send = hi ? e[s][w] : e[s | m][w];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+        if (hi) e[s][w] = recv;
+        else e[s | m][w] = recv;
+      }
+    }
+  }
+}
+
 // The work of one pair tile, in the order every role walks it.
 struct Item {
   int rb, ct;
@@ -849,42 +870,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = __all_sync(~0u, wait_on(&afull[a.idx], a.phase, wc, kPSiteDrainAcc)))) break;
         tc_fence_after();
       }
+      // Y = bf16(Y_res + Y_lr): Y_res = kDq acc (exact), Y_lr from tensor memory. Each
+      // 32-column chunk becomes four 16-byte pieces per row; a transpose within groups of
+      // four lanes (four rows) gives each lane one piece of each of the group's rows, so a
+      // store writes 64 contiguous bytes of 8 rows instead of 16 bytes of 32 rows.
       const int c0 = half * 128;
-      uint16_t* yrow = args.y + grow * args.n + it.ct * 256 + c0;
+      const int64_t row4 = static_cast<int64_t>(it.rb) * 256 + row_half + quarter * 32 + (lane & ~3);
+      uint16_t* ycol = args.y + it.ct * 256 + c0 + (lane & 3) * 8;
 #pragma unroll
       for (int c = 0; c < 128; c += 32) {
-        // Y = bf16(Y_res + Y_lr): Y_res = kDq acc (exact), Y_lr from tensor memory
-        float yv[8];
+        uint32_t v[32];
         if constexpr (T::s2) {
-          uint32_t v[32];
           tmem_ld32(tmem + lane_addr + a.idx * 256 + c0 + c, v);
           tmem_wait_ld();
-          if (row_ok) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-#pragma unroll
-              for (int k = 0; k < 8; ++k) yv[k] = acc[c + i + k] * kDq + __uint_as_float(v[i + k]);
-              *reinterpret_cast<uint4*>(yrow + c + i) =
-                  make_uint4(bf16x2(yv[0], yv[1]), bf16x2(yv[2], yv[3]), bf16x2(yv[4], yv[5]),
-                             bf16x2(yv[6], yv[7]));
-            }
-          }
-        } else if (row_ok) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) yv[k] = acc[c + i + k] * kDq;
-            *reinterpret_cast<uint4*>(yrow + c + i) =
-                make_uint4(bf16x2(yv[0], yv[1]), bf16x2(yv[2], yv[3]), bf16x2(yv[4], yv[5]),
-                           bf16x2(yv[6], yv[7]));
+          if (c == 96) {  // the stage-2 accumulator is read: free it before the last stores
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_n(aempty_lead + a.idx * 8, 1);
+            a.next(2);
           }
         }
-      }
-      if (T::s2) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster_n(aempty_lead + a.idx * 8, 1);
-        a.next(2);
+        uint32_t yw[4][4];  // four pieces of 8 columns, as BF16 pairs
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          float yv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if constexpr (T::s2) yv[k] = acc[c + i + k] * kDq + __uint_as_float(v[i + k]);
+            else yv[k] = acc[c + i + k] * kDq;
+          }
+          yw[i >> 3][0] = bf16x2(yv[0], yv[1]);
+          yw[i >> 3][1] = bf16x2(yv[2], yv[3]);
+          yw[i >> 3][2] = bf16x2(yv[4], yv[5]);
+          yw[i >> 3][3] = bf16x2(yv[6], yv[7]);
+        }
+        transpose4x4(yw, lane);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (row4 + j < args.b)
+            *reinterpret_cast<uint4*>(ycol + (row4 + j) * args.n + c) =
+                make_uint4(yw[j][0], yw[j][1], yw[j][2], yw[j][3]);
       }
     }
   }
